@@ -1,0 +1,142 @@
+"""Python front end of the fp64 CPU oracle (``oracle/oracle.c``).
+
+TEST INFRASTRUCTURE ONLY: the test suite, the entry module's smoke check and
+the benchmark's CPU-baseline leg are the only callers.  The CUDA library never
+imports this package, and this package imports nothing from the CUDA library.
+
+Arrays cross the boundary as C-contiguous float64 / int32 numpy arrays; the
+oracle itself does all of the arithmetic in C (see the citations there).
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import subprocess
+
+import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+SOURCE = os.path.join(_HERE, "oracle.c")
+LIBRARY = os.path.join(_HERE, "liboracle.so")
+
+
+def build(source: str = SOURCE, output: str = LIBRARY, extra_flags=()) -> str:
+    """Compile the oracle with gcc (no fast-math: IEEE double semantics)."""
+    cmd = ["gcc", "-O2", "-fopenmp", "-fPIC", "-shared", "-std=c11", *extra_flags,
+           source, "-o", output, "-lm"]
+    subprocess.run(cmd, check=True)
+    return output
+
+
+def _needs_build(lib: str, src: str) -> bool:
+    return not os.path.exists(lib) or os.path.getmtime(lib) < os.path.getmtime(src)
+
+
+_D = ctypes.POINTER(ctypes.c_double)
+_I = ctypes.POINTER(ctypes.c_int)
+
+
+def _dptr(a):
+    return None if a is None else a.ctypes.data_as(_D)
+
+
+def _iptr(a):
+    return None if a is None else a.ctypes.data_as(_I)
+
+
+def _f64(a):
+    return np.ascontiguousarray(np.asarray(a, dtype=np.float64))
+
+
+def _i32(a):
+    return None if a is None else np.ascontiguousarray(np.asarray(a, dtype=np.int32))
+
+
+class Oracle:
+    """ctypes handle on one compiled oracle library (the real one by default)."""
+
+    def __init__(self, library: str | None = None):
+        if library is None:
+            if _needs_build(LIBRARY, SOURCE):
+                build()
+            library = LIBRARY
+        self.lib = ctypes.CDLL(library)
+        L = self.lib
+        L.oracle_num_threads.restype = ctypes.c_int
+        L.oracle_causal_mask.argtypes = [_D, ctypes.c_int, ctypes.c_int]
+        L.oracle_sliding_window_mask.argtypes = [_D, ctypes.c_int, ctypes.c_int, ctypes.c_int]
+        L.oracle_attn_fwd.restype = ctypes.c_int
+        L.oracle_attn_fwd.argtypes = [_D, _D, _D, _D, _D] + [ctypes.c_int] * 6 + [
+            ctypes.c_double, ctypes.c_int, ctypes.c_int, ctypes.c_int, _I, _I, _I, ctypes.c_int]
+        L.oracle_decode.restype = ctypes.c_int
+        L.oracle_decode.argtypes = [_D, _D, _D, _D, _D] + [ctypes.c_int] * 5 + [_I]
+
+    def num_threads(self) -> int:
+        return int(self.lib.oracle_num_threads())
+
+    # -- mlx-arsenal "Attention" page mask builders ---------------------------------
+    def causal_mask(self, seq_len: int, offset: int = 0) -> np.ndarray:
+        """Additive mask of shape (1, 1, seq_len, offset + seq_len), 0 / -inf."""
+        out = np.empty((seq_len, offset + seq_len), dtype=np.float64)
+        self.lib.oracle_causal_mask(_dptr(out), seq_len, offset)
+        return out.reshape(1, 1, seq_len, offset + seq_len)
+
+    def sliding_window_mask(self, seq_len: int, window_size: int, offset: int = 0) -> np.ndarray:
+        out = np.empty((seq_len, offset + seq_len), dtype=np.float64)
+        self.lib.oracle_sliding_window_mask(_dptr(out), seq_len, window_size, offset)
+        return out.reshape(1, 1, seq_len, offset + seq_len)
+
+    # -- Tylo.jl "Primitives" page, attention! ----------------------------------------
+    def attn_fwd(self, Q, K, V, scale, causal=False, window=0, input_pos=0,
+                 k_lengths=None, q_lengths=None, rows=None, Sq=None):
+        """O (B,Hq,n,D) float64 and LSE (B,Hq,n) float64.
+
+        Q is (B, Hq, n, D).  When ``rows`` is given, Q holds only those query
+        rows (absolute indices into a sequence of ``Sq`` rows); otherwise Q is
+        the whole (B, Hq, Sq, D) tensor.
+        """
+        Q, K, V = _f64(Q), _f64(K), _f64(V)
+        B, Hq, n, D = Q.shape
+        Bk, Hkv, Sk, Dk = K.shape
+        assert Bk == B and Dk == D and V.shape == K.shape
+        rows_a = _i32(rows)
+        if rows_a is None:
+            Sq = n
+        else:
+            assert rows_a.shape == (n,) and Sq is not None
+        kl, ql = _i32(k_lengths), _i32(q_lengths)
+        O = np.empty((B, Hq, n, D), dtype=np.float64)
+        LSE = np.empty((B, Hq, n), dtype=np.float64)
+        rc = self.lib.oracle_attn_fwd(_dptr(O), _dptr(LSE), _dptr(Q), _dptr(K), _dptr(V),
+                                      B, Hq, Hkv, Sq, Sk, D, float(scale), int(causal),
+                                      int(window), int(input_pos), _iptr(kl), _iptr(ql),
+                                      _iptr(rows_a), n)
+        if rc != 0:
+            raise ValueError("oracle_attn_fwd rejected its arguments")
+        return O, LSE
+
+    # -- Tylo.jl "Primitives" page, decode_attention! ---------------------------------
+    def decode(self, Q, K, V, lengths):
+        """O (B,Hq,D) and LSE (B,Hq) float64; Q (B,Hq,D), K/V (B,Hkv,S_cap,D)."""
+        Q, K, V = _f64(Q), _f64(K), _f64(V)
+        B, Hq, D = Q.shape
+        _, Hkv, S_cap, _ = K.shape
+        ln = _i32(lengths)
+        O = np.empty((B, Hq, D), dtype=np.float64)
+        LSE = np.empty((B, Hq), dtype=np.float64)
+        rc = self.lib.oracle_decode(_dptr(O), _dptr(LSE), _dptr(Q), _dptr(K), _dptr(V),
+                                    B, Hq, Hkv, S_cap, D, _iptr(ln))
+        if rc != 0:
+            raise ValueError("oracle_decode rejected its arguments")
+        return O, LSE
+
+
+_DEFAULT: Oracle | None = None
+
+
+def default() -> Oracle:
+    """The oracle built from ``oracle/oracle.c`` (compiled on first use)."""
+    global _DEFAULT
+    if _DEFAULT is None:
+        _DEFAULT = Oracle()
+    return _DEFAULT

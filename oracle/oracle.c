@@ -1,0 +1,256 @@
+/*
+ * Plain fp64 CPU oracle for fused multi-head attention with GQA and for
+ * split-KV single-token decode.
+ *
+ * TEST INFRASTRUCTURE ONLY.  Nothing in the product path may link, load or
+ * call this file: only the test suite, the smoke check of the entry module and
+ * the CPU-baseline leg of the benchmark use it.  It shares no code, header,
+ * table or helper with the CUDA library.
+ *
+ * What it computes, and where each piece is defined:
+ *
+ *   - Tylo.jl "Primitives" page, entry `attention!`: O = softmax(Q K^T scale +
+ *     mask) V per (batch, query head), with GQA (Heads a multiple of
+ *     Heads_KV, entry `flex_attention!`), `input_pos` = absolute position of
+ *     the first query, `k_lengths`/`q_lengths` = per-batch valid lengths, and
+ *     the softmax statistics M/L saved for the backward.  We export them as
+ *     one number per row, LSE = M + ln L (natural log of the scaled scores).
+ *   - mlx-arsenal "Attention" page, entries `causal_mask` and
+ *     `sliding_window_mask`: additive masks of shape (1, 1, S, offset + S)
+ *     whose masked entries are -inf; the sliding window lets a query see at
+ *     most `window_size` previous positions, itself included.
+ *   - Tylo.jl "Primitives" page, entry `CausalMask`: a query sees keys at or
+ *     before its own position, positions being absolute (input_pos shifts the
+ *     queries).
+ *   - Tylo.jl "Primitives" page, entry `decode_attention!`: one query vector
+ *     per head and sequence against the first lengths[b] cached keys.  The
+ *     split into n_splits slices and their combine change only the rounding,
+ *     so the oracle computes the plain softmax over all valid keys.  Its scale
+ *     is the page's default qk_scale = 1/sqrt(Dk) (entry `flex_attention!`).
+ *
+ * Readings where the pages are silent (each one is listed in the design
+ * notes with its reason):
+ *   - GQA head map: query head h reads KV head h / (Hq / Hkv).
+ *   - valid lengths are prefixes: key j is valid iff j < k_lengths[b], query
+ *     row i is valid iff i < q_lengths[b].
+ *   - window w > 0 (always causal): key j is visible from absolute query
+ *     position p iff p - w < j <= p, i.e. at most w keys, itself included.
+ *   - a row with no visible key (invalid row, empty length, or every key cut)
+ *     has O = 0 and LSE = -inf.
+ *
+ * Precision: inputs are doubles (the harness widens the exact bf16 values),
+ * every product, sum, exp and log is done in double.
+ *
+ * Layouts (row-major, C order):
+ *   Q (B, Hq, n_rows, D)    -- n_rows query rows whose absolute row indices
+ *                              within 0..Sq-1 are rows[0..n_rows-1] (NULL:
+ *                              all Sq rows in order, n_rows == Sq)
+ *   K, V (B, Hkv, Sk, D)
+ *   O (B, Hq, n_rows, D), LSE (B, Hq, n_rows)
+ */
+#include <math.h>
+#include <stdlib.h>
+#include <string.h>
+#ifdef _OPENMP
+#include <omp.h>
+#endif
+
+/* Number of OpenMP threads an oracle call will use. */
+int oracle_num_threads(void) {
+#ifdef _OPENMP
+    return omp_get_max_threads();
+#else
+    return 1;
+#endif
+}
+
+/*
+ * mlx-arsenal "Attention" page, `causal_mask(seq_len, offset)`: the
+ * lower-triangular additive mask of shape (1, 1, seq_len, offset + seq_len);
+ * query row i (at position offset + i in a KV cache of offset + seq_len
+ * entries) sees keys 0..offset + i.  `out` holds seq_len * (offset + seq_len)
+ * doubles, each 0.0 or -inf.
+ */
+void oracle_causal_mask(double *out, int seq_len, int offset) {
+    const long n_kv = (long)offset + seq_len;
+    for (long i = 0; i < seq_len; ++i)
+        for (long j = 0; j < n_kv; ++j)
+            out[i * n_kv + j] = (j <= offset + i) ? 0.0 : -INFINITY;
+}
+
+/*
+ * mlx-arsenal "Attention" page, `sliding_window_mask(seq_len, window_size,
+ * offset)`: causal, and each position sees at most window_size previous
+ * positions including itself, i.e. keys offset+i-window_size+1 .. offset+i.
+ * Same shape and values as the causal mask.
+ */
+void oracle_sliding_window_mask(double *out, int seq_len, int window_size, int offset) {
+    const long n_kv = (long)offset + seq_len;
+    for (long i = 0; i < seq_len; ++i) {
+        const long pos = (long)offset + i;
+        for (long j = 0; j < n_kv; ++j) {
+            const int visible = (j <= pos) && (j > pos - window_size);
+            out[i * n_kv + j] = visible ? 0.0 : -INFINITY;
+        }
+    }
+}
+
+/*
+ * Additive mask row for absolute query row i of batch b: 0.0 where key j is
+ * visible, -inf elsewhere.  Combines the causal rule (Tylo `CausalMask`,
+ * absolute positions), the sliding window (mlx-arsenal
+ * `sliding_window_mask`), and the per-batch valid lengths of `attention!`.
+ */
+static void mask_row(double *m, long i, int Sk, int causal, int window, int input_pos,
+                     int k_len, int q_len) {
+    const long pos = (long)input_pos + i;
+    for (long j = 0; j < Sk; ++j) {
+        int visible = (i < q_len) && (j < k_len);
+        if (causal && j > pos) visible = 0;
+        if (window > 0 && j <= pos - window) visible = 0;
+        m[j] = visible ? 0.0 : -INFINITY;
+    }
+}
+
+/*
+ * Tylo.jl "Primitives" page, `attention!` (+ GQA rule of `flex_attention!`).
+ * For every batch b, query head hq and requested query row:
+ *   s_j   = scale * <Q_i, K_j> + mask_j          (explicit score row)
+ *   M     = max_j s_j,  L = sum_j exp(s_j - M)   (softmax statistics)
+ *   O_i   = sum_j (exp(s_j - M) / L) V_j
+ *   LSE_i = M + ln L
+ * Returns 0, or -1 on bad arguments.
+ */
+int oracle_attn_fwd(double *O, double *LSE, const double *Q, const double *K, const double *V,
+                    int B, int Hq, int Hkv, int Sq, int Sk, int D, double scale,
+                    int causal, int window, int input_pos,
+                    const int *k_lengths, const int *q_lengths,
+                    const int *rows, int n_rows) {
+    if (B < 0 || Hq <= 0 || Hkv <= 0 || Sq < 0 || Sk < 0 || D <= 0) return -1;
+    if (Hq % Hkv != 0) return -1;
+    if (window > 0 && !causal) return -1;
+    if (rows == NULL) n_rows = Sq;
+    const int group = Hq / Hkv;
+    const long total = (long)B * Hq * n_rows;
+    int bad = 0;
+
+#pragma omp parallel
+    {
+        double *score = (double *)malloc(sizeof(double) * (Sk > 0 ? Sk : 1));
+        double *mask = (double *)malloc(sizeof(double) * (Sk > 0 ? Sk : 1));
+        if (score == NULL || mask == NULL) {
+#pragma omp atomic write
+            bad = 1;
+        }
+#pragma omp for schedule(dynamic, 16)
+        for (long t = 0; t < total; ++t) {
+            if (score == NULL || mask == NULL) continue;
+            const long r = t % n_rows;
+            const long hq = (t / n_rows) % Hq;
+            const long b = t / ((long)n_rows * Hq);
+            const long i = rows ? rows[r] : r;
+            const long hkv = hq / group;
+            const int k_len = k_lengths ? k_lengths[b] : Sk;
+            const int q_len = q_lengths ? q_lengths[b] : Sq;
+
+            const double *q = Q + ((b * Hq + hq) * (long)n_rows + r) * D;
+            const double *Kb = K + (b * Hkv + hkv) * (long)Sk * D;
+            const double *Vb = V + (b * Hkv + hkv) * (long)Sk * D;
+            double *o = O + ((b * Hq + hq) * (long)n_rows + r) * D;
+
+            mask_row(mask, i, Sk, causal, window, input_pos, k_len, q_len);
+            double mx = -INFINITY;
+            for (long j = 0; j < Sk; ++j) {
+                double dot = 0.0;
+                for (int d = 0; d < D; ++d) dot += q[d] * Kb[j * D + d];
+                score[j] = scale * dot + mask[j];
+                if (score[j] > mx) mx = score[j];
+            }
+            for (int d = 0; d < D; ++d) o[d] = 0.0;
+            if (mx == -INFINITY) {
+                if (LSE) LSE[(b * Hq + hq) * (long)n_rows + r] = -INFINITY;
+                continue;
+            }
+            double l = 0.0;
+            for (long j = 0; j < Sk; ++j) {
+                score[j] = exp(score[j] - mx);
+                l += score[j];
+            }
+            for (long j = 0; j < Sk; ++j) {
+                const double p = score[j] / l;
+                if (p == 0.0) continue;
+                for (int d = 0; d < D; ++d) o[d] += p * Vb[j * D + d];
+            }
+            if (LSE) LSE[(b * Hq + hq) * (long)n_rows + r] = mx + log(l);
+        }
+        free(score);
+        free(mask);
+    }
+    return bad ? -1 : 0;
+}
+
+/*
+ * Tylo.jl "Primitives" page, `decode_attention!`: one query per (sequence b,
+ * query head hq) attends to cached keys 0..lengths[b]-1 of KV head
+ * hq / (Hq / Hkv), with scale 1/sqrt(D).
+ *   Q (B, Hq, D); K, V (B, Hkv, S_cap, D); O (B, Hq, D); LSE (B, Hq) or NULL.
+ * A sequence with lengths[b] == 0 yields O = 0 and LSE = -inf.
+ * Returns 0, or -1 on bad arguments (including a length above S_cap).
+ */
+int oracle_decode(double *O, double *LSE, const double *Q, const double *K, const double *V,
+                  int B, int Hq, int Hkv, int S_cap, int D, const int *lengths) {
+    if (B < 0 || Hq <= 0 || Hkv <= 0 || S_cap < 0 || D <= 0 || lengths == NULL) return -1;
+    if (Hq % Hkv != 0) return -1;
+    for (int b = 0; b < B; ++b)
+        if (lengths[b] < 0 || lengths[b] > S_cap) return -1;
+    const int group = Hq / Hkv;
+    const double scale = 1.0 / sqrt((double)D);
+    const long total = (long)B * Hq;
+    int bad = 0;
+
+#pragma omp parallel
+    {
+        double *score = (double *)malloc(sizeof(double) * (S_cap > 0 ? S_cap : 1));
+        if (score == NULL) {
+#pragma omp atomic write
+            bad = 1;
+        }
+#pragma omp for schedule(dynamic, 1)
+        for (long t = 0; t < total; ++t) {
+            if (score == NULL) continue;
+            const long hq = t % Hq;
+            const long b = t / Hq;
+            const long hkv = hq / group;
+            const int len = lengths[b];
+            const double *q = Q + (b * Hq + hq) * (long)D;
+            const double *Kb = K + (b * Hkv + hkv) * (long)S_cap * D;
+            const double *Vb = V + (b * Hkv + hkv) * (long)S_cap * D;
+            double *o = O + (b * Hq + hq) * (long)D;
+
+            for (int d = 0; d < D; ++d) o[d] = 0.0;
+            if (len == 0) {
+                if (LSE) LSE[b * Hq + hq] = -INFINITY;
+                continue;
+            }
+            double mx = -INFINITY;
+            for (long j = 0; j < len; ++j) {
+                double dot = 0.0;
+                for (int d = 0; d < D; ++d) dot += q[d] * Kb[j * D + d];
+                score[j] = scale * dot;
+                if (score[j] > mx) mx = score[j];
+            }
+            double l = 0.0;
+            for (long j = 0; j < len; ++j) {
+                score[j] = exp(score[j] - mx);
+                l += score[j];
+            }
+            for (long j = 0; j < len; ++j) {
+                const double p = score[j] / l;
+                for (int d = 0; d < D; ++d) o[d] += p * Vb[j * D + d];
+            }
+            if (LSE) LSE[b * Hq + hq] = mx + log(l);
+        }
+        free(score);
+    }
+    return bad ? -1 : 0;
+}

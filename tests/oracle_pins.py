@@ -1,0 +1,351 @@
+"""Pins for the fp64 oracle: facts the pages and the mathematics fix.
+
+Every pin takes an ``oracle.Oracle`` handle and raises ``AssertionError`` when
+the handle disagrees with the fact.  ``test_oracle_pins.py`` runs them on the
+real oracle; ``test_oracle_mutants.py`` runs them on copies of the oracle with
+a planted mistake and requires that each mistake fails at least one pin.
+
+None of these re-types the oracle's formula: each one checks a closed form, a
+count the pages state, an invariant, a hand-derived value (``golden/``), or a
+special case that a library routine (torch's scaled_dot_product_attention in
+float64) computes on its own.
+"""
+from __future__ import annotations
+
+import json
+import math
+import os
+
+import numpy as np
+import torch
+
+GOLDEN = os.path.join(os.path.dirname(os.path.abspath(__file__)), "golden")
+NEG_INF = -math.inf
+
+
+def _rng(seed):
+    return np.random.default_rng(seed)
+
+
+def _visible_count(p, window, k_len):
+    """Keys visible from absolute position p: interval [max(0,p-w+1), min(p, k_len-1)]."""
+    lo = max(0, p - window + 1) if window > 0 else 0
+    hi = min(p, k_len - 1)
+    return max(0, hi - lo + 1)
+
+
+# --------------------------------------------------------------------------------------
+# mlx-arsenal "Attention" page: causal_mask / sliding_window_mask
+# --------------------------------------------------------------------------------------
+
+def pin_causal_mask_shape_and_rows(orc):
+    """Shape (1,1,S,offset+S); entries 0/-inf; lower-triangular with a KV offset:
+    row i sees the offset cached keys plus queries 0..i, so offset+i+1 zeros that
+    form a prefix, and the last row sees every key."""
+    for S in range(1, 13):
+        for offset in range(0, 6):
+            m = orc.causal_mask(S, offset)
+            assert m.shape == (1, 1, S, offset + S)
+            m = m[0, 0]
+            assert np.all((m == 0.0) | (m == NEG_INF))
+            for i in range(S):
+                zeros = np.flatnonzero(m[i] == 0.0)
+                assert len(zeros) == offset + i + 1, (S, offset, i, len(zeros))
+                assert np.array_equal(zeros, np.arange(offset + i + 1))
+            assert np.all(m[S - 1] == 0.0)
+
+
+def pin_sliding_window_rows(orc):
+    """Each row sees at most window_size keys, itself included, ending on its own
+    position; a window at least as long as the sequence is the causal mask."""
+    for S in range(1, 11):
+        for offset in range(0, 4):
+            for w in range(1, S + offset + 2):
+                m = orc.sliding_window_mask(S, w, offset)
+                assert m.shape == (1, 1, S, offset + S)
+                m = m[0, 0]
+                assert np.all((m == 0.0) | (m == NEG_INF))
+                for i in range(S):
+                    zeros = np.flatnonzero(m[i] == 0.0)
+                    assert len(zeros) == min(w, offset + i + 1), (S, offset, w, i)
+                    assert zeros[-1] == offset + i
+                    assert np.all(np.diff(zeros) == 1)
+                if w >= S + offset:
+                    assert np.array_equal(m, orc.causal_mask(S, offset)[0, 0])
+
+
+# --------------------------------------------------------------------------------------
+# Tylo.jl "Primitives" page: attention!
+# --------------------------------------------------------------------------------------
+
+def pin_two_key_golden(orc):
+    """Hand-derived values in golden/two_key_softmax.json."""
+    with open(os.path.join(GOLDEN, "two_key_softmax.json")) as f:
+        g = json.load(f)
+    q = np.array(g["q"], dtype=np.float64)[None, None]          # (1,1,1,1)
+    k = np.array(g["k"], dtype=np.float64)[None, None]          # (1,1,2,1)
+    v = np.array(g["v"], dtype=np.float64)[None, None]
+    for case in g["cases"]:
+        O, L = orc.attn_fwd(q, k, v, math.log(3.0), causal=case["causal"],
+                            input_pos=case["input_pos"])
+        assert abs(O[0, 0, 0, 0] - case["O"][0]) < 1e-12, (case, O)
+        assert abs(L[0, 0, 0] - math.log(case["LSE_is_ln"])) < 1e-12, (case, L)
+
+
+def pin_probability_rows(orc):
+    """With V = identity the output rows are the probability rows: each sums to 1,
+    is >= 0, and is exactly 0 where the page-1 mask is -inf."""
+    rng = _rng(1)
+    for causal, window, offset, S in [(True, 0, 0, 7), (True, 0, 3, 6), (True, 3, 2, 8),
+                                      (False, 0, 0, 5), (True, 1, 4, 4)]:
+        Sk = offset + S
+        D = Sk
+        Q = rng.standard_normal((1, 2, S, D))
+        K = rng.standard_normal((1, 1, Sk, D))
+        V = np.eye(Sk)[None, None]
+        O, _ = orc.attn_fwd(Q, K, V, 0.7, causal=causal, window=window, input_pos=offset)
+        P = O
+        assert np.all(P >= 0.0)
+        assert np.allclose(P.sum(-1), 1.0, atol=1e-12, rtol=0)
+        if causal:
+            m = (orc.sliding_window_mask(S, window, offset) if window
+                 else orc.causal_mask(S, offset))[0, 0]
+            assert np.all(P[0, :, m == NEG_INF] == 0.0)
+            assert np.all(P[0, :, m == 0.0] > 0.0)
+
+
+def pin_constant_v(orc):
+    """A constant V row gives that row as output for every row that sees a key."""
+    rng = _rng(2)
+    B, Hq, Hkv, S, D = 2, 4, 2, 9, 5
+    vrow = rng.standard_normal(D)
+    Q = rng.standard_normal((B, Hq, S, D))
+    K = rng.standard_normal((B, Hkv, S, D))
+    V = np.broadcast_to(vrow, (B, Hkv, S, D)).copy()
+    for causal, window in [(False, 0), (True, 0), (True, 3)]:
+        O, _ = orc.attn_fwd(Q, K, V, 0.9, causal=causal, window=window)
+        assert np.allclose(O, vrow, atol=1e-12, rtol=0)
+
+
+def pin_causal_row0(orc):
+    """Causal, input_pos 0: query row 0 sees only key 0, so O[0] = V[0] exactly."""
+    rng = _rng(3)
+    Q = rng.standard_normal((1, 3, 6, 4))
+    K = rng.standard_normal((1, 3, 6, 4))
+    V = rng.standard_normal((1, 3, 6, 4))
+    O, L = orc.attn_fwd(Q, K, V, 0.5, causal=True)
+    assert np.array_equal(O[0, :, 0, :], V[0, :, 0, :])
+    s00 = 0.5 * np.einsum("hd,hd->h", Q[0, :, 0], K[0, :, 0])
+    assert np.allclose(L[0, :, 0], s00, atol=1e-12, rtol=0)
+
+
+def pin_uniform_attention(orc):
+    """K = 0 makes every visible score equal, so O_i is the mean of the visible V
+    rows and LSE_i = ln(number of visible keys); rows that see nothing give O = 0
+    and LSE = -inf.  Counts come from interval arithmetic on the definitions."""
+    rng = _rng(4)
+    B, Hq, Hkv, Sq, Sk, D = 3, 4, 2, 11, 14, 3
+    Q = rng.standard_normal((B, Hq, Sq, D))
+    K = np.zeros((B, Hkv, Sk, D))
+    V = rng.standard_normal((B, Hkv, Sk, D))
+    k_len = np.array([14, 5, 0], dtype=np.int32)
+    q_len = np.array([11, 7, 11], dtype=np.int32)
+    for causal, window, input_pos in [(False, 0, 0), (True, 0, 3), (True, 4, 2), (True, 1, 0)]:
+        O, L = orc.attn_fwd(Q, K, V, 1.3, causal=causal, window=window, input_pos=input_pos,
+                            k_lengths=k_len, q_lengths=q_len)
+        for b in range(B):
+            for hq in range(Hq):
+                hkv = hq // (Hq // Hkv)
+                for i in range(Sq):
+                    p = input_pos + i
+                    if i >= q_len[b]:
+                        n = 0
+                    elif causal:
+                        n = _visible_count(p, window, min(k_len[b], Sk))
+                        lo = max(0, p - window + 1) if window > 0 else 0
+                    else:
+                        n = int(min(k_len[b], Sk))
+                        lo = 0
+                    if n == 0:
+                        assert np.all(O[b, hq, i] == 0.0) and L[b, hq, i] == NEG_INF
+                        continue
+                    mean = V[b, hkv, lo:lo + n].mean(0)
+                    assert np.allclose(O[b, hq, i], mean, atol=1e-12, rtol=0), (b, hq, i)
+                    assert abs(L[b, hq, i] - math.log(n)) < 1e-12
+
+
+def pin_gqa_repeat(orc):
+    """GQA equals MHA on K/V heads repeated Hq/Hkv times (consecutive groups)."""
+    rng = _rng(5)
+    B, Hq, Hkv, Sq, Sk, D = 2, 6, 2, 5, 8, 4
+    Q = rng.standard_normal((B, Hq, Sq, D))
+    K = rng.standard_normal((B, Hkv, Sk, D))
+    V = rng.standard_normal((B, Hkv, Sk, D))
+    Kr = np.repeat(K, Hq // Hkv, axis=1)
+    Vr = np.repeat(V, Hq // Hkv, axis=1)
+    for causal, window, input_pos in [(False, 0, 0), (True, 0, 3), (True, 2, 3)]:
+        O1, L1 = orc.attn_fwd(Q, K, V, 0.8, causal=causal, window=window, input_pos=input_pos)
+        O2, L2 = orc.attn_fwd(Q, Kr, Vr, 0.8, causal=causal, window=window, input_pos=input_pos)
+        assert np.allclose(O1, O2, atol=1e-13, rtol=0)
+        assert np.allclose(L1, L2, atol=1e-13, rtol=0)
+
+
+def _sdpa(Q, K, V, scale, allowed):
+    q = torch.from_numpy(Q)
+    k = torch.from_numpy(K)
+    v = torch.from_numpy(V)
+    return torch.nn.functional.scaled_dot_product_attention(
+        q, k, v, attn_mask=torch.from_numpy(allowed), scale=scale).numpy()
+
+
+def pin_library_sdpa(orc):
+    """Against torch's scaled_dot_product_attention in float64 with the page-1
+    masks (causal_mask / sliding_window_mask with the KV offset) as the boolean
+    mask, on rows that see at least one key; K/V heads repeated for GQA."""
+    rng = _rng(6)
+    cases = [  # B, Hq, Hkv, S, offset, D, causal, window
+        (2, 4, 2, 9, 0, 16, False, 0),
+        (1, 4, 1, 7, 5, 8, True, 0),
+        (2, 2, 2, 12, 0, 8, True, 4),
+        (1, 6, 3, 6, 9, 32, True, 5),
+    ]
+    for B, Hq, Hkv, S, offset, D, causal, window in cases:
+        Sk = offset + S
+        Q = rng.standard_normal((B, Hq, S, D))
+        K = rng.standard_normal((B, Hkv, Sk, D))
+        V = rng.standard_normal((B, Hkv, Sk, D))
+        scale = 1.0 / math.sqrt(D)
+        O, _ = orc.attn_fwd(Q, K, V, scale, causal=causal, window=window, input_pos=offset)
+        if causal:
+            m = (orc.sliding_window_mask(S, window, offset) if window
+                 else orc.causal_mask(S, offset))[0, 0]
+            allowed = (m == 0.0)
+        else:
+            allowed = np.ones((S, Sk), dtype=bool)
+        ref = _sdpa(Q, np.repeat(K, Hq // Hkv, 1), np.repeat(V, Hq // Hkv, 1), scale, allowed)
+        assert np.allclose(O, ref, atol=1e-12, rtol=0), np.abs(O - ref).max()
+
+
+def pin_lse_matches_probabilities(orc):
+    """LSE is the log normaliser: P_ij = exp(s_ij - LSE_i) for the probabilities read
+    out with V = identity, and max_j s_ij <= LSE_i <= max_j s_ij + ln(n_i)."""
+    rng = _rng(7)
+    S, offset = 6, 2
+    Sk = S + offset
+    D = Sk
+    Q = rng.standard_normal((1, 1, S, D))
+    K = rng.standard_normal((1, 1, Sk, D))
+    P, L = orc.attn_fwd(Q, K, np.eye(Sk)[None, None], 1.1, causal=True, input_pos=offset)
+    s = 1.1 * (Q[0, 0] @ K[0, 0].T)
+    for i in range(S):
+        vis = np.arange(Sk) <= offset + i
+        assert np.all(P[0, 0, i, vis] > 0.0)
+        logp = np.log(P[0, 0, i, vis])
+        assert np.allclose(logp + L[0, 0, i], s[i, vis], atol=1e-12, rtol=0)
+        smax = s[i, vis].max()
+        assert smax - 1e-12 <= L[0, 0, i] <= smax + math.log(vis.sum()) + 1e-12
+
+
+def pin_lengths_are_prefixes(orc):
+    """k_lengths = L equals dropping keys L.. ; rows at or past q_lengths are O = 0,
+    LSE = -inf, and the rows before them are unchanged."""
+    rng = _rng(8)
+    B, Hq, Hkv, S, D = 2, 2, 1, 10, 6
+    Q = rng.standard_normal((B, Hq, S, D))
+    K = rng.standard_normal((B, Hkv, S, D))
+    V = rng.standard_normal((B, Hkv, S, D))
+    k_len = np.array([6, 10], dtype=np.int32)
+    q_len = np.array([10, 4], dtype=np.int32)
+    for causal in (False, True):
+        O, L = orc.attn_fwd(Q, K, V, 0.6, causal=causal, k_lengths=k_len, q_lengths=q_len)
+        for b in range(B):
+            Ob, Lb = orc.attn_fwd(Q[b:b + 1], K[b:b + 1, :, :k_len[b]], V[b:b + 1, :, :k_len[b]],
+                                  0.6, causal=causal)
+            ql = q_len[b]
+            assert np.allclose(O[b, :, :ql], Ob[0, :, :ql], atol=1e-13, rtol=0)
+            assert np.allclose(L[b, :, :ql], Lb[0, :, :ql], atol=1e-13, rtol=0)
+            assert np.all(O[b, :, ql:] == 0.0) and np.all(L[b, :, ql:] == NEG_INF)
+
+
+def pin_row_subset(orc):
+    """Computing a subset of query rows gives those rows of the full result."""
+    rng = _rng(9)
+    B, Hq, Hkv, S, D = 1, 4, 2, 13, 4
+    Q = rng.standard_normal((B, Hq, S, D))
+    K = rng.standard_normal((B, Hkv, S, D))
+    V = rng.standard_normal((B, Hkv, S, D))
+    rows = np.array([0, 5, 12, 7], dtype=np.int32)
+    O, L = orc.attn_fwd(Q, K, V, 0.4, causal=True, window=3, input_pos=2)
+    Os, Ls = orc.attn_fwd(Q[:, :, rows], K, V, 0.4, causal=True, window=3, input_pos=2,
+                          rows=rows, Sq=S)
+    assert np.array_equal(Os, O[:, :, rows]) and np.array_equal(Ls, L[:, :, rows])
+
+
+# --------------------------------------------------------------------------------------
+# Tylo.jl "Primitives" page: decode_attention!
+# --------------------------------------------------------------------------------------
+
+def pin_decode_is_last_row_of_prefill(orc):
+    """Single-token decode is causal attention of one query at absolute position
+    len-1 over the first len cached keys, with the default scale 1/sqrt(D)."""
+    rng = _rng(10)
+    B, Hq, Hkv, S_cap, D = 3, 4, 2, 12, 8
+    Q = rng.standard_normal((B, Hq, D))
+    K = rng.standard_normal((B, Hkv, S_cap, D))
+    V = rng.standard_normal((B, Hkv, S_cap, D))
+    lengths = np.array([12, 1, 7], dtype=np.int32)
+    O, L = orc.decode(Q, K, V, lengths)
+    for b in range(B):
+        n = int(lengths[b])
+        Op, Lp = orc.attn_fwd(Q[b:b + 1, :, None, :], K[b:b + 1], V[b:b + 1],
+                              1.0 / math.sqrt(D), causal=True, input_pos=n - 1)
+        assert np.allclose(O[b], Op[0, :, 0], atol=1e-13, rtol=0)
+        assert np.allclose(L[b], Lp[0, :, 0], atol=1e-13, rtol=0)
+
+
+def pin_decode_closed_forms(orc):
+    """Decode with K = 0 averages the first len V rows (LSE = ln len); a constant V
+    comes back unchanged; len = 0 gives O = 0, LSE = -inf; the scale is 1/sqrt(D)
+    (a single key with q.k = sqrt(D) has LSE exactly 1)."""
+    rng = _rng(11)
+    B, Hq, Hkv, S_cap, D = 3, 2, 1, 9, 16
+    Q = rng.standard_normal((B, Hq, D))
+    V = rng.standard_normal((B, Hkv, S_cap, D))
+    lengths = np.array([9, 3, 0], dtype=np.int32)
+    O, L = orc.decode(Q, np.zeros((B, Hkv, S_cap, D)), V, lengths)
+    for b in range(B):
+        n = int(lengths[b])
+        if n == 0:
+            assert np.all(O[b] == 0.0) and np.all(L[b] == NEG_INF)
+            continue
+        assert np.allclose(O[b], V[b, 0, :n].mean(0), atol=1e-12, rtol=0)
+        assert np.allclose(L[b], math.log(n), atol=1e-12, rtol=0)
+    vrow = rng.standard_normal(D)
+    Vc = np.broadcast_to(vrow, (B, Hkv, S_cap, D)).copy()
+    O, _ = orc.decode(Q, rng.standard_normal((B, Hkv, S_cap, D)), Vc, np.array([9, 4, 1]))
+    assert np.allclose(O, vrow, atol=1e-12, rtol=0)
+    # q = 1, k0 = 1/sqrt(D): q.k0 = sqrt(D), times the scale 1/sqrt(D) gives 1, and
+    # one visible key makes LSE equal to that score.
+    q1 = np.ones((1, 1, D))
+    k1 = np.zeros((1, 1, 2, D))
+    k1[0, 0, 0] = 1.0 / math.sqrt(D)
+    _, L1 = orc.decode(q1, k1, np.zeros((1, 1, 2, D)), np.array([1]))
+    assert abs(L1[0, 0] - 1.0) < 1e-12, L1
+
+
+PINS = [
+    pin_causal_mask_shape_and_rows,
+    pin_sliding_window_rows,
+    pin_two_key_golden,
+    pin_probability_rows,
+    pin_constant_v,
+    pin_causal_row0,
+    pin_uniform_attention,
+    pin_gqa_repeat,
+    pin_library_sdpa,
+    pin_lse_matches_probabilities,
+    pin_lengths_are_prefixes,
+    pin_row_subset,
+    pin_decode_is_last_row_of_prefill,
+    pin_decode_closed_forms,
+]

@@ -1,0 +1,66 @@
+"""Each planted mistake in a copy of the oracle must fail at least one pin.
+
+The mistakes are the plausible ones: an off-by-one in a mask, the window read
+as w+1 keys, a wrong GQA head map, a dropped scale, K and V swapped, a dropped
+term in the log-sum-exp, ignored lengths or input_pos, a missing
+normalisation, the wrong default decode scale.  Copies are built in a
+temporary directory from ``oracle/oracle.c`` with one textual substitution
+each; the real oracle is never modified.
+"""
+import pytest
+
+import oracle
+from oracle_pins import PINS
+
+MUTANTS = {
+    "causal_off_by_one": ("if (causal && j > pos) visible = 0;",
+                          "if (causal && j >= pos) visible = 0;"),
+    "window_w_plus_1": ("if (window > 0 && j <= pos - window) visible = 0;",
+                        "if (window > 0 && j < pos - window) visible = 0;"),
+    "gqa_modulo_map": ("const long hkv = hq / group;\n            const int k_len",
+                       "const long hkv = hq % Hkv;\n            const int k_len"),
+    "scale_dropped": ("score[j] = scale * dot + mask[j];", "score[j] = dot + mask[j];"),
+    "k_v_swapped": ("dot += q[d] * Kb[j * D + d];\n                score[j] = scale * dot + mask[j];",
+                    "dot += q[d] * Vb[j * D + d];\n                score[j] = scale * dot + mask[j];"),
+    "decode_k_v_swapped": ("dot += q[d] * Kb[j * D + d];\n                score[j] = scale * dot;",
+                           "dot += q[d] * Vb[j * D + d];\n                score[j] = scale * dot;"),
+    "lse_missing_max": ("LSE[(b * Hq + hq) * (long)n_rows + r] = mx + log(l);",
+                        "LSE[(b * Hq + hq) * (long)n_rows + r] = log(l);"),
+    "q_lengths_ignored": ("int visible = (i < q_len) && (j < k_len);", "int visible = (j < k_len);"),
+    "k_lengths_ignored": ("int visible = (i < q_len) && (j < k_len);", "int visible = (i < q_len);"),
+    "input_pos_ignored": ("const long pos = (long)input_pos + i;\n    for (long j = 0; j < Sk; ++j) {",
+                          "const long pos = i;\n    for (long j = 0; j < Sk; ++j) {"),
+    "not_normalised": ("const double p = score[j] / l;\n                if (p == 0.0)",
+                       "const double p = score[j];\n                if (p == 0.0)"),
+    "decode_scale": ("const double scale = 1.0 / sqrt((double)D);", "const double scale = 1.0 / (double)D;"),
+    "decode_lse_missing_max": ("if (LSE) LSE[b * Hq + hq] = mx + log(l);", "if (LSE) LSE[b * Hq + hq] = log(l);"),
+    "decode_gqa_modulo": ("const long hkv = hq / group;\n            const int len",
+                          "const long hkv = hq % Hkv;\n            const int len"),
+    "page1_causal_strict": ("out[i * n_kv + j] = (j <= offset + i) ? 0.0 : -INFINITY;",
+                            "out[i * n_kv + j] = (j < offset + i) ? 0.0 : -INFINITY;"),
+    "page1_window_wide": ("const int visible = (j <= pos) && (j > pos - window_size);",
+                          "const int visible = (j <= pos) && (j >= pos - window_size);"),
+}
+
+
+@pytest.fixture(scope="module")
+def source():
+    with open(oracle.SOURCE) as f:
+        return f.read()
+
+
+@pytest.mark.parametrize("name", sorted(MUTANTS))
+def test_mutant_is_caught(name, source, tmp_path):
+    old, new = MUTANTS[name]
+    assert source.count(old) == 1, f"mutation site for {name} not unique in oracle.c"
+    src = tmp_path / f"{name}.c"
+    src.write_text(source.replace(old, new))
+    lib = oracle.build(str(src), str(tmp_path / f"lib{name}.so"))
+    mutant = oracle.Oracle(lib)
+    failed = []
+    for pin in PINS:
+        try:
+            pin(mutant)
+        except AssertionError:
+            failed.append(pin.__name__)
+    assert failed, f"no pin catches the planted mistake {name}"
