@@ -1,0 +1,105 @@
+"""Thin ctypes binding over ``libgqa_attn.so`` (C ABI in ``include/gqa_attn.h``).
+
+Argument marshalling only: every step of the attention path runs in the CUDA
+kernels behind the C entry points.  The functions take torch tensors for
+convenience, pass their device pointers and the current CUDA stream, and raise
+``AttnError`` on a non-OK status.  There is no fallback: if the library is
+missing or fails to load, importing this module raises.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIBRARY = os.path.join(_HERE, "libgqa_attn.so")
+
+if not os.path.exists(LIBRARY):
+    raise ImportError(f"{LIBRARY} is not built; run `python -m gqa_attention_flash_b200.build`")
+
+lib = ctypes.CDLL(LIBRARY)
+
+ATTN_OK = 0
+STATUS = {0: "ATTN_OK", 1: "ATTN_ERR_NULL", 2: "ATTN_ERR_INVALID", 3: "ATTN_ERR_UNSUPPORTED",
+          4: "ATTN_ERR_CUDA", 5: "ATTN_ERR_TIMEOUT", 6: "ATTN_ERR_DEVICE_BOUNDS"}
+
+_p = ctypes.c_void_p
+_i = ctypes.c_int
+_f = ctypes.c_float
+
+lib.attn_fwd.restype = _i
+lib.attn_fwd.argtypes = [_p, _p, _p, _p, _p] + [_i] * 6 + [_f, _i, _i, _i, _p, _p]
+lib.attn_fwd_varlen.restype = _i
+lib.attn_fwd_varlen.argtypes = [_p, _p, _p, _p, _p] + [_i] * 6 + [_f, _i, _i, _i, _p, _p, _p]
+lib.attn_decode.restype = _i
+lib.attn_decode.argtypes = [_p, _p, _p, _p, _p, _i, _p] + [_i] * 5
+lib.attn_status_string.restype = ctypes.c_char_p
+lib.attn_status_string.argtypes = [_i]
+lib.attn_last_device_status.restype = _i
+lib.attn_last_device_status.argtypes = [_p]
+lib.attn_check_bounded_wait.restype = _i
+lib.attn_check_bounded_wait.argtypes = [_i, _p]
+
+
+class AttnError(RuntimeError):
+    def __init__(self, status: int, where: str):
+        self.status = status
+        super().__init__(f"{where}: {lib.attn_status_string(status).decode()}")
+
+
+def _ptr(t):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream):
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return ctypes.c_void_p(stream.cuda_stream)
+
+
+def _check(rc: int, where: str):
+    if rc != ATTN_OK:
+        raise AttnError(rc, where)
+
+
+def status_string(status: int) -> str:
+    return lib.attn_status_string(status).decode()
+
+
+def attn_fwd(O, Q, K, V, LSE, scale, causal=False, window=0, input_pos=0, k_lengths=None,
+             q_lengths=None, stream=None):
+    """Fill O (B,Hq,Sq,D) bf16 and LSE (B,Hq,Sq) fp32 (or None) in place.
+
+    Shapes are read from the tensors: Q (B,Hq,Sq,D), K/V (B,Hkv,Sk,D).  Calls
+    ``attn_fwd_varlen`` when q_lengths is given, else ``attn_fwd``.
+    """
+    B, Hq, Sq, D = Q.shape
+    _, Hkv, Sk, _ = K.shape
+    args = [_ptr(O), _ptr(Q), _ptr(K), _ptr(V), _ptr(LSE), B, Hq, Hkv, Sq, Sk, D, float(scale),
+            int(causal), int(window), int(input_pos), _ptr(k_lengths)]
+    if q_lengths is not None:
+        rc = lib.attn_fwd_varlen(*args, _ptr(q_lengths), _stream(stream))
+        _check(rc, "attn_fwd_varlen")
+    else:
+        rc = lib.attn_fwd(*args, _stream(stream))
+        _check(rc, "attn_fwd")
+
+
+def attn_decode(O, Q, K, V, lengths, n_splits=8, stream=None):
+    """Fill O (B,Hq,D) bf16 in place; Q (B,Hq,D), K/V caches (B,Hkv,S_cap,D)."""
+    B, Hq, D = Q.shape
+    _, Hkv, S_cap, _ = K.shape
+    rc = lib.attn_decode(_ptr(O), _ptr(Q), _ptr(K), _ptr(V), _ptr(lengths), int(n_splits),
+                         _stream(stream), B, Hq, Hkv, S_cap, D)
+    _check(rc, "attn_decode")
+
+
+def last_device_status(stream=None) -> int:
+    """Synchronise the stream and return (and clear) the device status word."""
+    return lib.attn_last_device_status(_stream(stream))
+
+
+def check_bounded_wait(limit_us: int, stream=None):
+    _check(lib.attn_check_bounded_wait(int(limit_us), _stream(stream)), "attn_check_bounded_wait")

@@ -1,0 +1,224 @@
+// attn_api.cu -- the library's C ABI (declared in include/gqa_attn.h):
+// host-side argument validation, TMA descriptor encoding, the per-device status
+// word, and the decode workspace.
+#include <cmath>
+#include <cstdint>
+#include <cstring>
+#include <mutex>
+
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include "internal.h"
+#include "sm100_ptx.cuh"
+
+namespace gqa {
+
+__device__ int g_status = 0;
+
+size_t decode_workspace_floats(int B, int Hq, int n_splits, int D);
+
+namespace {
+
+typedef CUresult (*EncodeTiledFn)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *,
+                                  const cuuint64_t *, const cuuint64_t *, const cuuint32_t *,
+                                  const cuuint32_t *, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                  CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+    static EncodeTiledFn fn = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        void *ptr = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) ==
+                cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<EncodeTiledFn>(ptr);
+    });
+    return fn;
+}
+
+bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+}  // namespace
+
+attn_status_t make_tmap_bf16_3d(CUtensorMap *map, const void *base, uint64_t D, uint64_t rows,
+                                uint64_t outer, uint32_t box_rows) {
+    EncodeTiledFn fn = encode_fn();
+    if (!fn) return ATTN_ERR_CUDA;
+    const cuuint64_t dims[3] = {D, rows > 0 ? rows : 1, outer > 0 ? outer : 1};
+    const cuuint64_t strides[2] = {D * 2, D * 2 * (rows > 0 ? rows : 1)};
+    const cuuint32_t box[3] = {64, box_rows, 1};
+    const cuuint32_t estr[3] = {1, 1, 1};
+    CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void *>(base), dims,
+                    strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                    CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS ? ATTN_OK : ATTN_ERR_INVALID;
+}
+
+namespace {
+
+__global__ void wait_probe_kernel(uint64_t limit_ns) {
+    __shared__ __align__(8) uint64_t bar;
+    __shared__ int abort_flag;
+    const uint32_t b = smem_u32(&bar);
+    if (threadIdx.x == 0) {
+        mbar_init(b, 1);
+        abort_flag = 0;
+        fence_mbar_init();
+    }
+    __syncthreads();
+    // Nobody arrives on `bar`: the bounded wait must give up and record the status.
+    warp_wait(b, 0, &abort_flag, limit_ns);
+    __syncthreads();
+}
+
+}  // namespace
+
+attn_status_t launch_wait_probe(int limit_us, cudaStream_t stream) {
+    wait_probe_kernel<<<1, 32, 0, stream>>>(static_cast<uint64_t>(limit_us) * 1000ull);
+    return cudaGetLastError() == cudaSuccess ? ATTN_OK : ATTN_ERR_CUDA;
+}
+
+}  // namespace gqa
+
+using namespace gqa;
+
+namespace {
+
+attn_status_t validate_fwd(void *O, const void *Q, const void *K, const void *V, float *LSE, int B,
+                           int Hq, int Hkv, int Sq, int Sk, int D, float scale, int causal,
+                           int window, int input_pos) {
+    if (B < 0 || Sq < 0 || Sk < 0 || Hq < 1 || Hkv < 1 || input_pos < 0 || window < 0)
+        return ATTN_ERR_INVALID;
+    if (Hq % Hkv != 0) return ATTN_ERR_INVALID;
+    if (causal != 0 && causal != 1) return ATTN_ERR_INVALID;
+    if (window > 0 && !causal) return ATTN_ERR_INVALID;
+    if (!(scale > 0.f) || !std::isfinite(scale)) return ATTN_ERR_INVALID;
+    if (D != 64 && D != 128) return ATTN_ERR_UNSUPPORTED;
+    const long long rows_q = (long long)B * Hq * Sq, rows_k = (long long)B * Hkv * Sk;
+    if (rows_q > 0 && (!O || !Q)) return ATTN_ERR_NULL;
+    if (rows_q > 0 && Sk > 0 && (!K || !V)) return ATTN_ERR_NULL;
+    if (!aligned16(O) || !aligned16(Q) || !aligned16(K) || !aligned16(V) || !aligned16(LSE))
+        return ATTN_ERR_INVALID;
+    // TMA coordinates are 32-bit and each dimension must stay below 2^32 elements.
+    if ((long long)B * Hq > 0x7fffffffll || (long long)B * Hkv > 0x7fffffffll)
+        return ATTN_ERR_INVALID;
+    (void)rows_k;
+    (void)LSE;
+    return ATTN_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+attn_status_t attn_fwd_varlen(void *O, const void *Q, const void *K, const void *V, float *LSE,
+                              int B, int Hq, int Hkv, int Sq, int Sk, int D, float scale,
+                              int causal, int window, int input_pos, const int32_t *k_lengths,
+                              const int32_t *q_lengths, void *stream) {
+    attn_status_t st =
+        validate_fwd(O, Q, K, V, LSE, B, Hq, Hkv, Sq, Sk, D, scale, causal, window, input_pos);
+    if (st != ATTN_OK) return st;
+    if ((long long)B * Hq * Sq == 0) return ATTN_OK;
+    FwdArgs a;
+    a.O = O;
+    a.Q = Q;
+    a.K = K;
+    a.V = V;
+    a.LSE = LSE;
+    a.k_lengths = k_lengths;
+    a.q_lengths = q_lengths;
+    a.B = B;
+    a.Hq = Hq;
+    a.Hkv = Hkv;
+    a.Sq = Sq;
+    a.Sk = Sk;
+    a.D = D;
+    a.scale = scale;
+    a.causal = causal;
+    a.window = window;
+    a.input_pos = input_pos;
+    if (Sk == 0) {
+        // No key at all: every row is empty.  The kernel handles k_end = 0 but
+        // needs a valid K/V tensor map; use the query tensor as a stand-in.
+        a.K = Q;
+        a.V = Q;
+        a.Sk = 0;
+    }
+    return launch_fwd(a, static_cast<cudaStream_t>(stream));
+}
+
+attn_status_t attn_fwd(void *O, const void *Q, const void *K, const void *V, float *LSE, int B,
+                       int Hq, int Hkv, int Sq, int Sk, int D, float scale, int causal, int window,
+                       int input_pos, const int32_t *k_lengths, void *stream) {
+    return attn_fwd_varlen(O, Q, K, V, LSE, B, Hq, Hkv, Sq, Sk, D, scale, causal, window,
+                           input_pos, k_lengths, nullptr, stream);
+}
+
+attn_status_t attn_decode(void *O, const void *Q, const void *K, const void *V,
+                          const int32_t *lengths, int n_splits, void *stream, int B, int Hq,
+                          int Hkv, int S_cap, int D) {
+    if (B < 0 || Hq < 1 || Hkv < 1 || S_cap < 0 || n_splits < 1 || n_splits > 64)
+        return ATTN_ERR_INVALID;
+    if (Hq % Hkv != 0 || Hq / Hkv > 16) return ATTN_ERR_INVALID;
+    if (D != 64 && D != 128) return ATTN_ERR_UNSUPPORTED;
+    if (B == 0) return ATTN_OK;
+    if (!O || !Q || !lengths) return ATTN_ERR_NULL;
+    if (S_cap > 0 && (!K || !V)) return ATTN_ERR_NULL;
+    if (!aligned16(O) || !aligned16(Q) || !aligned16(K) || !aligned16(V) ||
+        (reinterpret_cast<uintptr_t>(lengths) & 3u))
+        return ATTN_ERR_INVALID;
+    if ((long long)B * Hkv > 0x7fffffffll) return ATTN_ERR_INVALID;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    const size_t bytes = decode_workspace_floats(B, Hq, n_splits, D) * sizeof(float);
+    void *ws = nullptr;
+    if (cudaMallocAsync(&ws, bytes, s) != cudaSuccess) return ATTN_ERR_CUDA;
+    DecodeArgs a;
+    a.O = O;
+    a.Q = Q;
+    a.K = S_cap > 0 ? K : Q;
+    a.V = S_cap > 0 ? V : Q;
+    a.lengths = lengths;
+    a.n_splits = n_splits;
+    a.B = B;
+    a.Hq = Hq;
+    a.Hkv = Hkv;
+    a.S_cap = S_cap;
+    a.D = D;
+    a.workspace = static_cast<float *>(ws);
+    attn_status_t st = launch_decode(a, s);
+    if (cudaFreeAsync(ws, s) != cudaSuccess && st == ATTN_OK) st = ATTN_ERR_CUDA;
+    return st;
+}
+
+const char *attn_status_string(attn_status_t status) {
+    switch (status) {
+        case ATTN_OK: return "ATTN_OK";
+        case ATTN_ERR_NULL: return "ATTN_ERR_NULL: a required pointer is NULL";
+        case ATTN_ERR_INVALID: return "ATTN_ERR_INVALID: inconsistent sizes, flags or alignment";
+        case ATTN_ERR_UNSUPPORTED: return "ATTN_ERR_UNSUPPORTED: head size not built (64, 128)";
+        case ATTN_ERR_CUDA: return "ATTN_ERR_CUDA: a CUDA call failed";
+        case ATTN_ERR_TIMEOUT: return "ATTN_ERR_TIMEOUT: a bounded device wait ran out";
+        case ATTN_ERR_DEVICE_BOUNDS: return "ATTN_ERR_DEVICE_BOUNDS: a length exceeded its tensor";
+    }
+    return "unknown attn_status_t";
+}
+
+attn_status_t attn_last_device_status(void *stream) {
+    if (cudaStreamSynchronize(static_cast<cudaStream_t>(stream)) != cudaSuccess)
+        return ATTN_ERR_CUDA;
+    int v = 0;
+    if (cudaMemcpyFromSymbol(&v, g_status, sizeof(int)) != cudaSuccess) return ATTN_ERR_CUDA;
+    const int zero = 0;
+    if (cudaMemcpyToSymbol(g_status, &zero, sizeof(int)) != cudaSuccess) return ATTN_ERR_CUDA;
+    return static_cast<attn_status_t>(v);
+}
+
+attn_status_t attn_check_bounded_wait(int limit_us, void *stream) {
+    if (limit_us < 1 || limit_us > 2000000) return ATTN_ERR_INVALID;
+    return launch_wait_probe(limit_us, static_cast<cudaStream_t>(stream));
+}
+
+}  // extern "C"

@@ -1,0 +1,43 @@
+// internal.h -- declarations shared by the library's translation units.
+#pragma once
+
+#include <cstdint>
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include "gqa_attn.h"
+
+namespace gqa {
+
+// Encode a 3-D bf16 tensor map over a row-major (outer, rows, D) tensor with
+// a (64, box_rows, 1) box and 128-byte swizzle; out-of-range rows read as 0.
+attn_status_t make_tmap_bf16_3d(CUtensorMap *map, const void *base, uint64_t D, uint64_t rows,
+                                uint64_t outer, uint32_t box_rows);
+
+struct FwdArgs {
+    void *O;
+    const void *Q, *K, *V;
+    float *LSE;
+    const int32_t *k_lengths, *q_lengths;
+    int B, Hq, Hkv, Sq, Sk, D;
+    float scale;
+    int causal, window, input_pos;
+};
+
+struct DecodeArgs {
+    void *O;
+    const void *Q, *K, *V;
+    const int32_t *lengths;
+    int n_splits;
+    int B, Hq, Hkv, S_cap, D;
+    float *workspace;  // B * Hq * n_splits * (D + 1) floats
+};
+
+attn_status_t launch_fwd(const FwdArgs &a, cudaStream_t stream);
+attn_status_t launch_decode(const DecodeArgs &a, cudaStream_t stream);
+attn_status_t launch_wait_probe(int limit_us, cudaStream_t stream);
+
+// Bounded-wait limit used by the attention kernels (nanoseconds of global time).
+constexpr uint64_t kWaitLimitNs = 2000000000ull;
+
+}  // namespace gqa

@@ -1,0 +1,152 @@
+/*
+ * gqa_attn.h -- C ABI of libgqa_attn.so: fused multi-head attention forward
+ * with grouped-query attention (GQA) and split-KV single-token decode, written
+ * for NVIDIA B200 (sm_100a).
+ *
+ * Conventions shared by every entry point
+ * ---------------------------------------
+ *  - Tensors are caller-owned DEVICE buffers (allocated by the caller, e.g.
+ *    with PyTorch), dense and row-major (C order).  Q, K, V and O hold bf16
+ *    values (raw 16-bit storage); LSE holds float32; lengths hold int32.
+ *    Every tensor base address must be 16-byte aligned.
+ *  - `stream` is a cudaStream_t passed as void* (NULL = the legacy default
+ *    stream).  Calls are asynchronous: they validate their arguments on the
+ *    host, enqueue kernels on `stream` and return.  The library never
+ *    synchronises a stream except in attn_last_device_status().
+ *  - Errors detectable on the host are returned before anything is enqueued:
+ *    ATTN_ERR_NULL for a NULL required pointer, ATTN_ERR_INVALID for
+ *    inconsistent sizes or flags, ATTN_ERR_UNSUPPORTED for a head size the
+ *    library was not built for, ATTN_ERR_CUDA when a CUDA call fails.
+ *  - Errors found on the device (a bounded wait that ran out, a length
+ *    outside the tensor) are recorded in a per-device status word and read
+ *    back with attn_last_device_status().  Kernels never trap.
+ *  - Query head h reads key/value head h / (Hq / Hkv): consecutive groups of
+ *    Hq / Hkv query heads share one K/V head (GQA; Heads must be a multiple of
+ *    Heads_KV -- Tylo.jl "Primitives" page, entry `flex_attention!`).
+ */
+#ifndef GQA_ATTN_H
+#define GQA_ATTN_H
+
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    ATTN_OK = 0,
+    ATTN_ERR_NULL = 1,          /* a required pointer is NULL */
+    ATTN_ERR_INVALID = 2,       /* sizes / flags inconsistent, misaligned pointer */
+    ATTN_ERR_UNSUPPORTED = 3,   /* head size D not built (built: 64, 128) */
+    ATTN_ERR_CUDA = 4,          /* a CUDA runtime / driver call failed */
+    ATTN_ERR_TIMEOUT = 5,       /* device: a bounded wait ran out, kernel gave up */
+    ATTN_ERR_DEVICE_BOUNDS = 6  /* device: a length exceeded the tensor, clamped */
+} attn_status_t;
+
+/*
+ * attn_fwd -- fused attention forward, O = softmax(Q K^T * scale + mask) V.
+ *
+ * Defined by: Tylo.jl "Primitives" page, entry `attention!` (fused MHA with
+ * GQA; keywords causal, input_pos = absolute position of the first query,
+ * k_lengths / q_lengths = optional per-batch valid lengths; the softmax
+ * statistics M/L are saved for the backward; Float32 accumulation), the
+ * causal rule of entry `CausalMask` (a query sees keys at or before its own
+ * absolute position), and the sliding window of the mlx-arsenal "Attention"
+ * page, entry `sliding_window_mask` (at most window_size keys, the query's
+ * own position included).
+ *
+ *   O     [out] bf16 (B, Hq, Sq, D)
+ *   Q     [in]  bf16 (B, Hq, Sq, D)
+ *   K, V  [in]  bf16 (B, Hkv, Sk, D)
+ *   LSE   [out] float32 (B, Hq, Sq) or NULL (statistics not saved).
+ *         LSE = M + ln L in natural-log units of the scaled scores, where
+ *         M = max_j s_j and L = sum_j exp(s_j - M) over the visible keys.
+ *   scale       multiplies Q K^T (the pages' default is 1/sqrt(D)).
+ *   causal      0 or 1.  Key j is visible from query row i only if
+ *               j <= input_pos + i.
+ *   window      0 = no window; w > 0 (requires causal) keeps only keys with
+ *               input_pos + i - w < j <= input_pos + i.
+ *   input_pos   >= 0, absolute position of query row 0.
+ *   k_lengths   int32 (B,) device array or NULL (= Sk): keys j >= k_lengths[b]
+ *               are invisible.  Values above Sk are clamped to Sk and flagged
+ *               ATTN_ERR_DEVICE_BOUNDS; negative values count as 0.
+ *   Sizes: B, Sq, Sk >= 0; Hq, Hkv >= 1, Hq % Hkv == 0; D in {64, 128}.
+ *
+ * A query row that sees no key (k_length 0, or every key cut by the masks)
+ * gets O = 0 and LSE = -inf.  Key/value rows at positions >= k_lengths[b]
+ * contribute exactly zero, whatever they hold.
+ */
+attn_status_t attn_fwd(void *O, const void *Q, const void *K, const void *V, float *LSE,
+                       int B, int Hq, int Hkv, int Sq, int Sk, int D, float scale,
+                       int causal, int window, int input_pos,
+                       const int32_t *k_lengths, void *stream);
+
+/*
+ * attn_fwd_varlen -- attn_fwd plus per-batch valid query lengths.
+ *
+ * Same definition and arguments as attn_fwd, with q_lengths an int32 (B,)
+ * device array or NULL (= Sq): query rows i >= q_lengths[b] are invalid and
+ * get O = 0 and LSE = -inf (Tylo.jl "Primitives" page, entry `attention!`,
+ * keyword q_lengths).  attn_fwd(...) is attn_fwd_varlen(..., q_lengths=NULL).
+ */
+attn_status_t attn_fwd_varlen(void *O, const void *Q, const void *K, const void *V, float *LSE,
+                              int B, int Hq, int Hkv, int Sq, int Sk, int D, float scale,
+                              int causal, int window, int input_pos,
+                              const int32_t *k_lengths, const int32_t *q_lengths,
+                              void *stream);
+
+/*
+ * attn_decode -- split-KV (Flash-Decoding) attention of one new query token per
+ * head and sequence against a KV cache.
+ *
+ * Defined by: Tylo.jl "Primitives" page, entry `decode_attention!` (one query
+ * vector per head and sequence, the KV cache processed in n_splits parallel
+ * slices, lengths = valid KV length per sequence); scale is the page's default
+ * qk_scale = 1/sqrt(D) (entry `flex_attention!`).  Slice s of sequence b
+ * covers keys [s*C, min((s+1)*C, lengths[b])) with C = 64 * ceil(ceil(
+ * lengths[b]/64) / n_splits); each slice yields a partial output and its
+ * log-sum-exp, and a second kernel merges the slices by their log-sum-exp.
+ *
+ *   O        [out] bf16 (B, Hq, D)
+ *   Q        [in]  bf16 (B, Hq, D)
+ *   K, V     [in]  bf16 caches (B, Hkv, S_cap, D)
+ *   lengths  [in]  int32 (B,) device array, required.  Values above S_cap are
+ *                  clamped and flagged ATTN_ERR_DEVICE_BOUNDS; values <= 0
+ *                  give O = 0 for that sequence.
+ *   n_splits 1..64.
+ *   Sizes: B >= 0; Hq, Hkv >= 1, Hq % Hkv == 0, Hq / Hkv <= 16;
+ *          S_cap >= 0; D in {64, 128}.
+ *
+ * The per-slice partial results live in a workspace of
+ * B * Hq * n_splits * (D + 1) floats that the call allocates and frees in
+ * stream order (cudaMallocAsync / cudaFreeAsync on `stream`).
+ */
+attn_status_t attn_decode(void *O, const void *Q, const void *K, const void *V,
+                          const int32_t *lengths, int n_splits, void *stream,
+                          int B, int Hq, int Hkv, int S_cap, int D);
+
+/* Human-readable name of a status code (static storage, never NULL). */
+const char *attn_status_string(attn_status_t status);
+
+/*
+ * attn_last_device_status -- synchronise `stream`, then return and clear the
+ * status word that kernels of this library set on the current device
+ * (ATTN_OK if none did).  Returns ATTN_ERR_CUDA if the synchronisation failed.
+ */
+attn_status_t attn_last_device_status(void *stream);
+
+/*
+ * attn_check_bounded_wait -- diagnostic for the library's bounded waits.
+ * Launches one block that waits on a barrier nobody completes, with a limit
+ * of `limit_us` microseconds (1..2000000), through the same wait routine the
+ * attention kernels use.  The kernel gives up, records ATTN_ERR_TIMEOUT in
+ * the device status word and returns; read it with attn_last_device_status.
+ * No page defines this; it exists to test the failure path without a hang.
+ */
+attn_status_t attn_check_bounded_wait(int limit_us, void *stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* GQA_ATTN_H */

@@ -1,0 +1,102 @@
+"""CUDA prefill path (attn_fwd / attn_fwd_varlen through the C ABI) against the
+fp64 oracle, element by element on the same seeded bf16 inputs."""
+import numpy as np
+import pytest
+import torch
+
+from gpu_common import compare, gpu_prefill, oracle_prefill, sample_rows
+from gqa_attention_flash_b200 import workloads as W
+
+pytestmark = pytest.mark.gpu
+
+
+def test_tiny_config_full(orc):
+    """The tiny causal GQA workload, every output element."""
+    w = W.TINY
+    x = W.make_prefill(w)
+    O, L = gpu_prefill(x.Q, x.K, x.V, w.scale, w.causal)
+    Or, Lr = oracle_prefill(orc, x.Q, x.K, x.V, w.scale, w.causal)
+    compare(O, L, Or, Lr, what="tiny")
+
+
+CASES = [
+    # B, Hq, Hkv, Sq, Sk, D, causal, window, input_pos, ragged
+    (1, 2, 1, 300, 300, 64, True, 0, 0, False),
+    (2, 4, 2, 300, 333, 128, False, 0, 0, False),
+    (2, 4, 2, 257, 700, 128, True, 0, 443, False),
+    (1, 4, 1, 520, 520, 128, True, 100, 0, False),
+    (2, 8, 2, 390, 390, 64, True, 130, 0, True),
+    (2, 3, 3, 129, 600, 128, False, 0, 0, True),
+    (1, 2, 2, 1, 257, 128, True, 0, 256, False),
+    (3, 2, 1, 200, 200, 128, True, 1, 0, False),
+    (1, 4, 4, 384, 384, 128, True, 0, 0, False),
+]
+
+
+@pytest.mark.parametrize("case", CASES, ids=[str(c) for c in CASES])
+def test_ragged_tiles(orc, case):
+    B, Hq, Hkv, Sq, Sk, D, causal, window, input_pos, ragged = case
+    Q, K, V = W.random_prefill(hash(case) % 1000, B, Hq, Hkv, Sq, Sk, D)
+    kl = ql = None
+    if ragged:
+        g = torch.Generator().manual_seed(7)
+        kl = torch.randint(1, Sk + 1, (B,), generator=g).to(torch.int32)
+        ql = torch.randint(1, Sq + 1, (B,), generator=g).to(torch.int32)
+    scale = 1.0 / np.sqrt(D)
+    O, L = gpu_prefill(Q, K, V, scale, causal, window, input_pos, kl, ql)
+    Or, Lr = oracle_prefill(orc, Q, K, V, scale, causal, window, input_pos, kl, ql)
+    compare(O, L, Or, Lr, what=str(case))
+
+
+def test_lse_optional(orc):
+    Q, K, V = W.random_prefill(3, 1, 2, 1, 200, 200, 128)
+    O, _ = gpu_prefill(Q, K, V, 0.1, True, want_lse=False)
+    Or, Lr = oracle_prefill(orc, Q, K, V, 0.1, True)
+    compare(O, None, Or, Lr, what="no LSE")
+
+
+def test_edge_cases(orc):
+    """Empty lengths, rows past q_len, keys cut entirely, Sk = 0."""
+    B, Hq, Hkv, S, D = 4, 2, 1, 200, 128
+    Q, K, V = W.random_prefill(11, B, Hq, Hkv, S, S, D)
+    kl = torch.tensor([0, 200, 5, 130], dtype=torch.int32)
+    ql = torch.tensor([200, 0, 200, 129], dtype=torch.int32)
+    for causal, window, input_pos in [(False, 0, 0), (True, 0, 0), (True, 3, 0), (True, 0, 150)]:
+        O, L = gpu_prefill(Q, K, V, 0.09, causal, window, input_pos, kl, ql)
+        Or, Lr = oracle_prefill(orc, Q, K, V, 0.09, causal, window, input_pos, kl, ql)
+        compare(O, L, Or, Lr, what=f"edge {causal} {window} {input_pos}")
+    Qe = Q[:, :, :7].contiguous()
+    Ke = torch.zeros(B, Hkv, 0, D, dtype=torch.bfloat16)
+    O, L = gpu_prefill(Qe, Ke, Ke, 0.1, False)
+    assert torch.all(O == 0) and torch.all(torch.isneginf(L))
+
+
+def test_nan_beyond_k_lengths_ignored(orc):
+    """Key/value rows past k_lengths may hold NaN; they must not leak."""
+    B, Hq, Hkv, S, D = 2, 2, 1, 300, 128
+    Q, K, V = W.random_prefill(12, B, Hq, Hkv, S, S, D)
+    kl = torch.tensor([157, 300], dtype=torch.int32)
+    Kp, Vp = K.clone(), V.clone()
+    Kp[0, :, 157:] = float("nan")
+    Vp[0, :, 157:] = float("nan")
+    O, L = gpu_prefill(Q, Kp, Vp, 0.09, True, 0, 0, kl)
+    Or, Lr = oracle_prefill(orc, Q, K, V, 0.09, True, 0, 0, kl)
+    compare(O, L, Or, Lr, what="nan past k_len")
+
+
+@pytest.mark.parametrize("name", ["llm", "window", "image"])
+def test_full_size_sampled(orc, name):
+    """Full-size workloads in the benchmark's launch configuration, compared on
+    sampled query rows (all batches and heads) including tile and mask edges."""
+    w = W.PREFILL_WORKLOADS[name]
+    x = W.make_prefill(w)
+    O, L = gpu_prefill(x.Q, x.K, x.V, w.scale, w.causal, w.window, w.input_pos, x.k_lengths,
+                       x.q_lengths)
+    extra = []
+    if x.k_lengths is not None:
+        for v in x.k_lengths.tolist():
+            extra += [v - 1, v, v - w.window, v - w.window + 1]
+    rows = sample_rows(w.Sq, 5, n_random=12, extra=extra)
+    Or, Lr = oracle_prefill(orc, x.Q, x.K, x.V, w.scale, w.causal, w.window, w.input_pos,
+                            x.k_lengths, x.q_lengths, rows=rows)
+    compare(O, L, Or, Lr, rows=rows, what=name)
