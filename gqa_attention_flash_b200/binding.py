@@ -23,7 +23,8 @@ lib = ctypes.CDLL(LIBRARY)
 
 ATTN_OK = 0
 STATUS = {0: "ATTN_OK", 1: "ATTN_ERR_NULL", 2: "ATTN_ERR_INVALID", 3: "ATTN_ERR_UNSUPPORTED",
-          4: "ATTN_ERR_CUDA", 5: "ATTN_ERR_TIMEOUT", 6: "ATTN_ERR_DEVICE_BOUNDS"}
+          4: "ATTN_ERR_CUDA", 5: "ATTN_ERR_TIMEOUT", 6: "ATTN_ERR_DEVICE_BOUNDS",
+          7: "ATTN_ERR_SCRATCH_LIMIT"}
 
 _p = ctypes.c_void_p
 _i = ctypes.c_int
@@ -35,6 +36,8 @@ lib.attn_fwd_varlen.restype = _i
 lib.attn_fwd_varlen.argtypes = [_p, _p, _p, _p, _p] + [_i] * 6 + [_f, _i, _i, _i, _p, _p, _p]
 lib.attn_decode.restype = _i
 lib.attn_decode.argtypes = [_p, _p, _p, _p, _p, _i, _p] + [_i] * 5
+lib.attn_decode_noalloc.restype = _i
+lib.attn_decode_noalloc.argtypes = [_p, _p, _p, _p, _p, _i, _p] + [_i] * 5
 lib.attn_status_string.restype = ctypes.c_char_p
 lib.attn_status_string.argtypes = [_i]
 lib.attn_last_device_status.restype = _i
@@ -94,6 +97,17 @@ def attn_decode(O, Q, K, V, lengths, n_splits=8, stream=None):
     rc = lib.attn_decode(_ptr(O), _ptr(Q), _ptr(K), _ptr(V), _ptr(lengths), int(n_splits),
                          _stream(stream), B, Hq, Hkv, S_cap, D)
     _check(rc, "attn_decode")
+
+
+def attn_decode_noalloc(O, Q, K, V, lengths, n_splits=8, stream=None):
+    """attn_decode without any allocation: the workspace lives in the library's
+    fixed 16 MiB device array (for callers that cannot allocate device memory;
+    calls that overlap on the GPU share that array and must be ordered)."""
+    B, Hq, D = Q.shape
+    _, Hkv, S_cap, _ = K.shape
+    rc = lib.attn_decode_noalloc(_ptr(O), _ptr(Q), _ptr(K), _ptr(V), _ptr(lengths),
+                                 int(n_splits), _stream(stream), B, Hq, Hkv, S_cap, D)
+    _check(rc, "attn_decode_noalloc")
 
 
 def last_device_status(stream=None) -> int:

@@ -202,6 +202,9 @@ const char *attn_status_string(attn_status_t status) {
         case ATTN_ERR_CUDA: return "ATTN_ERR_CUDA: a CUDA call failed";
         case ATTN_ERR_TIMEOUT: return "ATTN_ERR_TIMEOUT: a bounded device wait ran out";
         case ATTN_ERR_DEVICE_BOUNDS: return "ATTN_ERR_DEVICE_BOUNDS: a length exceeded its tensor";
+        case ATTN_ERR_SCRATCH_LIMIT:
+            return "ATTN_ERR_SCRATCH_LIMIT: workspace exceeds the 16 MiB fixed array of "
+                   "attn_decode_noalloc";
     }
     return "unknown attn_status_t";
 }

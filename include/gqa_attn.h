@@ -40,7 +40,8 @@ typedef enum {
     ATTN_ERR_UNSUPPORTED = 3,   /* head size D not built (built: 64, 128) */
     ATTN_ERR_CUDA = 4,          /* a CUDA runtime / driver call failed */
     ATTN_ERR_TIMEOUT = 5,       /* device: a bounded wait ran out, kernel gave up */
-    ATTN_ERR_DEVICE_BOUNDS = 6  /* device: a length exceeded the tensor, clamped */
+    ATTN_ERR_DEVICE_BOUNDS = 6, /* device: a length exceeded the tensor, clamped */
+    ATTN_ERR_SCRATCH_LIMIT = 7  /* attn_decode_noalloc: workspace above its fixed array */
 } attn_status_t;
 
 /*
@@ -124,6 +125,36 @@ attn_status_t attn_fwd_varlen(void *O, const void *Q, const void *K, const void 
 attn_status_t attn_decode(void *O, const void *Q, const void *K, const void *V,
                           const int32_t *lengths, int n_splits, void *stream,
                           int B, int Hq, int Hkv, int S_cap, int D);
+
+/*
+ * attn_decode_noalloc -- attn_decode for callers that cannot allocate device
+ * memory.  The pages have no counterpart: it is attn_decode with a different
+ * home for the per-slice workspace.
+ *
+ * Who needs it: attn_decode calls cudaMallocAsync / cudaFreeAsync on every
+ * call.  A serving loop that reserves all of its device memory up front and
+ * forbids allocation afterwards (an allocation can fail once the memory is
+ * spoken for, and its latency is not bounded), or a program whose device
+ * memory belongs to another allocator, cannot let the library allocate.  This
+ * entry point allocates nothing: it runs the same kernels with the workspace
+ * in a fixed 16 MiB device array compiled into the library.
+ *
+ * Arguments, layouts, results and errors: as attn_decode, plus
+ * ATTN_ERR_SCRATCH_LIMIT, returned before anything is enqueued, when the
+ * workspace B * Hq * n_splits * (D + 4) * 4 bytes exceeds 16 MiB
+ * (16777216 bytes; e.g. B 64, Hq 32, n_splits 8, D 128 needs 8.65 MB).
+ *
+ * Sharing rules: every GPU that loads the library holds the 16 MiB array until
+ * the process exits, and all calls on one device share it.  Calls that can
+ * overlap on the GPU (other streams, unordered host threads) race on it; issue
+ * them on one stream or otherwise order them.  The array keeps the last call's
+ * contents; nothing in it needs to start at zero.  The first call on a device,
+ * made while that device is current, looks up the array's device address
+ * (cudaGetSymbolAddress); make that first call before any stream capture.
+ */
+attn_status_t attn_decode_noalloc(void *O, const void *Q, const void *K, const void *V,
+                                  const int32_t *lengths, int n_splits, void *stream,
+                                  int B, int Hq, int Hkv, int S_cap, int D);
 
 /* Human-readable name of a status code (static storage, never NULL). */
 const char *attn_status_string(attn_status_t status);
