@@ -119,7 +119,7 @@ attn_status_t attn_fwd_varlen(void *O, const void *Q, const void *K, const void 
  *          S_cap >= 0; D in {64, 128}.
  *
  * The per-slice partial results live in a workspace of
- * B * Hq * n_splits * (D + 1) floats that the call allocates and frees in
+ * B * Hq * n_splits * (D + 4) floats that the call allocates and frees in
  * stream order (cudaMallocAsync / cudaFreeAsync on `stream`).
  */
 attn_status_t attn_decode(void *O, const void *Q, const void *K, const void *V,
