@@ -1,23 +1,29 @@
 // attn_fwd.cu -- fused GQA attention forward for sm_100a.
 //
-// Computes, per (batch b, query head hq, 128-row query tile), the rows of
-// O = softmax(Q K^T * scale + mask) V and their log-sum-exp, as defined on the
-// Tylo.jl "Primitives" page (entry `attention!`: fused MHA with GQA, causal,
-// input_pos, k_lengths / q_lengths, saved softmax statistics M/L, Float32
-// accumulation) with the sliding window of the mlx-arsenal "Attention" page
-// (entry `sliding_window_mask`).
+// Computes the rows of O = softmax(Q K^T * scale + mask) V and their
+// log-sum-exp, as defined on the Tylo.jl "Primitives" page (entry `attention!`:
+// fused MHA with GQA, causal, input_pos, k_lengths / q_lengths, saved softmax
+// statistics M/L, Float32 accumulation) with the sliding window of the
+// mlx-arsenal "Attention" page (entry `sliding_window_mask`).
 //
-// One CTA per (query tile, hq, b); 6 warps with fixed roles:
-//   warps 0-3  softmax: one thread per query row (TMEM lane), online softmax
-//              in fp32 in the exp2 domain, P written back to TMEM as bf16,
-//              lazy O rescaling, epilogue O / L -> bf16 and LSE.
-//   warp 4     TMA producer: Q once, then K_j / V_j into an NS-stage ring.
-//   warp 5     MMA issuer (one thread): S_j = Q K_j^T into one of two TMEM S
-//              buffers, O += P_j V_j with P read from TMEM; owns the TMEM
-//              allocation.
-// Only the KV tiles that hold a visible key are visited (whole-tile skipping
-// for causal / window / length masks, Tylo `flex_attention!` keyword
-// block_sparse); the per-element mask is applied on boundary tiles only.
+// One CTA per (pair of 128-row query tiles, query head, batch).  The two query
+// tiles share every K/V tile the CTA loads, and their softmax runs alternate
+// with the tensor core (while warpgroup 0 turns S0 into P0, the tensor core
+// computes P1 V and the next S1, and the other way round).  12 warps:
+//   warps 0-3  softmax of query tile 0 (one row per thread = TMEM lane)
+//   warps 4-7  softmax of query tile 1
+//   warp 8     TMA producer: Q0/Q1 once, then K_j / V_j into an NS-stage ring
+//   warp 9     MMA issuer (one thread) and TMEM owner:
+//              S_t = Q_t K_j^T (smem x smem -> TMEM), O_t += P_t V_j (P_t read
+//              from TMEM, written there by the softmax over S_t)
+//   warps 10-11 idle
+// The block launches with 168 registers per thread; the producer warpgroup
+// (warps 8-11) drops to 56 and the two softmax warpgroups rise to 224
+// (128 * 56 + 256 * 224 = 384 * 168).
+// TMEM (512 columns): S0 | S1 | O0 | O1.  Each query tile visits only the KV
+// tiles that hold a key it can see (whole-tile skipping for causal, window and
+// length masks -- Tylo `flex_attention!` keyword block_sparse); the
+// per-element mask is applied on boundary tiles only.
 #include <cuda_bf16.h>
 
 #include "internal.h"
@@ -27,35 +33,42 @@ namespace gqa {
 
 namespace {
 
-constexpr int BM = 128;  // query rows per tile (= TMEM lanes)
-constexpr int BN = 128;  // keys per KV tile
-constexpr int kThreads = 192;
+constexpr int BM = 128;         // query rows per query tile (= TMEM lanes)
+constexpr int BN = 128;         // keys per KV tile
+constexpr int kTiles = 2;       // query tiles per CTA
+constexpr int kWarpTma = 8;
+constexpr int kWarpMma = 9;
+constexpr int kThreads = 384;
+constexpr int kLaunchRegs = 168;     // per thread at launch (checked on the host)
+constexpr uint32_t kProducerRegs = 56;
+constexpr uint32_t kSoftmaxRegs = 224;
+static_assert(128 * kProducerRegs + 256 * kSoftmaxRegs <= kThreads * kLaunchRegs,
+              "register split must use exactly the launch allocation");
 
 template <int D>
 struct FwdCfg {
     static constexpr int NS = (D == 128) ? 2 : 4;  // K/V ring depth
     static constexpr int NBOX = D / 64;             // 64-column TMA boxes per row
-    static constexpr int BOX_Q = BM * 128;           // bytes of one Q box
-    static constexpr int BOX_KV = BN * 128;          // bytes of one K or V box
-    static constexpr int Q_BYTES = BM * D * 2;
-    static constexpr int KV_BYTES = BN * D * 2;
+    static constexpr int BOX = 128 * 128;            // bytes of one (128 rows x 64 cols) box
+    static constexpr int Q_BYTES = BM * D * 2;       // one query tile
+    static constexpr int KV_BYTES = BN * D * 2;      // one K or V tile
     static constexpr int OFF_Q = 0;
-    static constexpr int OFF_K = OFF_Q + Q_BYTES;
+    static constexpr int OFF_K = OFF_Q + kTiles * Q_BYTES;
     static constexpr int OFF_V = OFF_K + NS * KV_BYTES;
     static constexpr int OFF_BAR = OFF_V + NS * KV_BYTES;
-    // barriers: q_full, k_full[NS], v_full[NS], kv_empty[NS], s_full[2], p_full[2], o_done
     static constexpr int BAR_Q = 0;
     static constexpr int BAR_KFULL = 1;
     static constexpr int BAR_VFULL = 1 + NS;
     static constexpr int BAR_EMPTY = 1 + 2 * NS;
-    static constexpr int BAR_SFULL = 1 + 3 * NS;
-    static constexpr int BAR_PFULL = 3 + 3 * NS;
-    static constexpr int BAR_ODONE = 5 + 3 * NS;
-    static constexpr int N_BARS = 6 + 3 * NS;
+    static constexpr int BAR_SFULL = 1 + 3 * NS;   // [2]
+    static constexpr int BAR_PFULL = 3 + 3 * NS;   // [2]
+    static constexpr int BAR_ODONE = 5 + 3 * NS;   // [2]
+    static constexpr int N_BARS = 7 + 3 * NS;
     static constexpr int OFF_MISC = OFF_BAR + N_BARS * 8;  // tmem slot, abort flag
     static constexpr int SMEM_BYTES = OFF_MISC + 16 + 1024;  // + alignment slack
     static constexpr uint32_t TMEM_COLS = 512;
-    static constexpr uint32_t O_COL = 256;  // S buffers at columns 0 and 128
+    __host__ __device__ static constexpr uint32_t s_col(int t) { return t * BN; }
+    __host__ __device__ static constexpr uint32_t o_col(int t) { return 2 * BN + t * D; }
 };
 
 struct FwdParams {
@@ -63,7 +76,7 @@ struct FwdParams {
     float *LSE;
     const int32_t *k_lengths;
     const int32_t *q_lengths;
-    int B, Hq, Hkv, Sq, Sk, group, n_qtiles;
+    int B, Hq, Hkv, Sq, Sk, group, n_pairs;
     float scale_log2;  // scale * log2(e)
     int causal, window, input_pos;
     uint64_t wait_limit_ns;
@@ -87,22 +100,21 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
 
-    // ---- which tile: heaviest causal query tiles first, sibling heads adjacent ----
+    // ---- which work: heaviest causal query-tile pairs first, sibling heads adjacent ----
     int bid = blockIdx.x;
     const int hq = bid % p.Hq;
     bid /= p.Hq;
     const int b = bid % p.B;
     bid /= p.B;
-    const int qt = p.n_qtiles - 1 - bid;
+    const int pair = p.n_pairs - 1 - bid;
     const int hkv = hq / p.group;
-    const int q0 = qt * BM;
 
-    // ---- visible KV range of this tile (step a1: whole-tile skipping) ----
+    // ---- visible KV tile range of each query tile (step a1: whole-tile skipping) ----
     int k_end = p.Sk, q_end = p.Sq;
     if (p.k_lengths) {
         int kl = p.k_lengths[b];
         if (kl > p.Sk) {
-            if (threadIdx.x == 0 && hq == 0 && qt == 0) record_status(ATTN_ERR_DEVICE_BOUNDS);
+            if (threadIdx.x == 0 && hq == 0 && pair == 0) record_status(ATTN_ERR_DEVICE_BOUNDS);
             kl = p.Sk;
         }
         k_end = kl > 0 ? kl : 0;
@@ -110,23 +122,38 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (p.q_lengths) {
         int ql = p.q_lengths[b];
         if (ql > p.Sq) {
-            if (threadIdx.x == 0 && hq == 0 && qt == 0) record_status(ATTN_ERR_DEVICE_BOUNDS);
+            if (threadIdx.x == 0 && hq == 0 && pair == 0) record_status(ATTN_ERR_DEVICE_BOUNDS);
             ql = p.Sq;
         }
         q_end = ql > 0 ? ql : 0;
     }
-    int n_tiles = 0, t_begin = 0, q_last = q0;
-    if (q0 < q_end && k_end > 0) {
-        q_last = min(q0 + BM - 1, q_end - 1);
-        long long hi = k_end;
-        if (p.causal) hi = min(hi, (long long)p.input_pos + q_last + 1);
-        long long lo = 0;
-        if (p.window > 0) lo = max(0ll, (long long)p.input_pos + q0 - p.window + 1);
-        if (hi > lo) {
-            t_begin = static_cast<int>(lo / BN);
-            n_tiles = static_cast<int>((hi + BN - 1) / BN) - t_begin;
+    // Tile t (0, 1) covers rows [q0_t, q0_t + 128) and sees KV tiles [lo_t, hi_t).
+    int lo0 = 0, hi0 = 0, lo1 = 0, hi1 = 0, ql0 = 0, ql1 = 0;
+#pragma unroll
+    for (int t = 0; t < kTiles; ++t) {
+        const int q0 = (pair * kTiles + t) * BM;
+        int lo_t = 0, hi_t = 0, qlast = q0;
+        if (q0 < q_end && k_end > 0) {
+            qlast = min(q0 + BM - 1, q_end - 1);
+            long long hi = k_end;
+            if (p.causal) hi = min(hi, (long long)p.input_pos + qlast + 1);
+            long long lo = 0;
+            if (p.window > 0) lo = max(0ll, (long long)p.input_pos + q0 - p.window + 1);
+            if (hi > lo) {
+                lo_t = static_cast<int>(lo / BN);
+                hi_t = static_cast<int>((hi + BN - 1) / BN);
+            }
         }
+        if (t == 0) { lo0 = lo_t; hi0 = hi_t; ql0 = qlast; }
+        else { lo1 = lo_t; hi1 = hi_t; ql1 = qlast; }
     }
+    const bool act0 = hi0 > lo0, act1 = hi1 > lo1;
+    const int u_lo = act0 ? (act1 ? min(lo0, lo1) : lo0) : lo1;
+    const int u_hi = act0 ? (act1 ? max(hi0, hi1) : hi0) : hi1;
+    const int n_u = (act0 || act1) ? u_hi - u_lo : 0;  // KV tiles the CTA loads
+#define TILE_LO(t) ((t) ? lo1 : lo0)
+#define TILE_HI(t) ((t) ? hi1 : hi0)
+#define USES(t, u) ((u) >= TILE_LO(t) && (u) < TILE_HI(t))
 
     // ---- set-up ----
     if (threadIdx.x == 0) {
@@ -136,15 +163,15 @@ __global__ void __launch_bounds__(kThreads, 1)
             mbar_init(bar(C::BAR_VFULL + s), 1);
             mbar_init(bar(C::BAR_EMPTY + s), 1);
         }
-        for (int s = 0; s < 2; ++s) {
-            mbar_init(bar(C::BAR_SFULL + s), 1);
-            mbar_init(bar(C::BAR_PFULL + s), BM);
+        for (int t = 0; t < kTiles; ++t) {
+            mbar_init(bar(C::BAR_SFULL + t), 1);
+            mbar_init(bar(C::BAR_PFULL + t), BM);
+            mbar_init(bar(C::BAR_ODONE + t), 1);
         }
-        mbar_init(bar(C::BAR_ODONE), 1);
         *abort_flag = 0;
         fence_mbar_init();
     }
-    if (warp == 5) {
+    if (warp == kWarpMma) {
         tmem_alloc(smem_u32(tmem_slot), C::TMEM_COLS);
         tmem_relinquish();
     }
@@ -153,130 +180,156 @@ __global__ void __launch_bounds__(kThreads, 1)
     tc_fence_after();
     const uint32_t tmem = *tmem_slot;
 
-    if (n_tiles > 0 && warp == 4) {
+    if (warp >= 8) {
+      regs_dec<kProducerRegs>();
+      if (warp == kWarpTma) {
         // ===================== TMA producer =====================
-        if (lane == 0) {
+        if (lane == 0 && n_u > 0) {
             prefetch_tensormap(&tmQ);
             prefetch_tensormap(&tmK);
             prefetch_tensormap(&tmV);
-            mbar_arrive_expect_tx(bar(C::BAR_Q), C::Q_BYTES);
-            for (int c = 0; c < C::NBOX; ++c)
-                tma_load_3d(sbase + C::OFF_Q + c * C::BOX_Q, &tmQ, bar(C::BAR_Q), c * 64, q0,
-                            b * p.Hq + hq);
-            for (int it = 0; it < n_tiles; ++it) {
-                const int st = it % C::NS;
-                const int use = it / C::NS;
+            const int nq = (act0 ? 1 : 0) + (act1 ? 1 : 0);
+            mbar_arrive_expect_tx(bar(C::BAR_Q), nq * C::Q_BYTES);
+#pragma unroll
+            for (int t = 0; t < kTiles; ++t) {
+                if (!(t ? act1 : act0)) continue;
+                for (int c = 0; c < C::NBOX; ++c)
+                    tma_load_3d(sbase + C::OFF_Q + t * C::Q_BYTES + c * C::BOX, &tmQ, bar(C::BAR_Q),
+                                c * 64, (pair * kTiles + t) * BM, b * p.Hq + hq);
+            }
+            for (int g = 0; g < n_u; ++g) {
+                const int st = g % C::NS;
+                const int use = g / C::NS;
                 if (use > 0 &&
                     !mbar_wait(bar(C::BAR_EMPTY + st), (use - 1) & 1, abort_flag, p.wait_limit_ns))
                     break;
-                const int kv_row = (t_begin + it) * BN;
+                const int kv_row = (u_lo + g) * BN;
                 mbar_arrive_expect_tx(bar(C::BAR_KFULL + st), C::KV_BYTES);
                 for (int c = 0; c < C::NBOX; ++c)
-                    tma_load_3d(sbase + C::OFF_K + st * C::KV_BYTES + c * C::BOX_KV, &tmK,
+                    tma_load_3d(sbase + C::OFF_K + st * C::KV_BYTES + c * C::BOX, &tmK,
                                 bar(C::BAR_KFULL + st), c * 64, kv_row, b * p.Hkv + hkv);
                 mbar_arrive_expect_tx(bar(C::BAR_VFULL + st), C::KV_BYTES);
                 for (int c = 0; c < C::NBOX; ++c)
-                    tma_load_3d(sbase + C::OFF_V + st * C::KV_BYTES + c * C::BOX_KV, &tmV,
+                    tma_load_3d(sbase + C::OFF_V + st * C::KV_BYTES + c * C::BOX, &tmV,
                                 bar(C::BAR_VFULL + st), c * 64, kv_row, b * p.Hkv + hkv);
             }
         }
-    } else if (n_tiles > 0 && warp == 5) {
+      } else if (warp == kWarpMma) {
         // ===================== MMA issuer =====================
-        if (lane == 0) {
+        if (lane == 0 && n_u > 0) {
             constexpr uint32_t idS = idesc_bf16_f32(BM, BN, 0, 0);
             constexpr uint32_t idO = idesc_bf16_f32(BM, D, 0, 1);
-            auto issue_s = [&](int it) -> bool {
-                const int st = it % C::NS;
-                const int buf = it & 1;
-                if (!mbar_wait(bar(C::BAR_KFULL + st), (it / C::NS) & 1, abort_flag,
+            auto issue_s = [&](int t, int u) -> bool {
+                const int g = u - u_lo;
+                const int st = g % C::NS;
+                if (!mbar_wait(bar(C::BAR_KFULL + st), (g / C::NS) & 1, abort_flag,
                                p.wait_limit_ns))
                     return false;
                 tc_fence_after();
-                const uint32_t qa = sbase + C::OFF_Q;
+                const uint32_t qa = sbase + C::OFF_Q + t * C::Q_BYTES;
                 const uint32_t ka = sbase + C::OFF_K + st * C::KV_BYTES;
 #pragma unroll
                 for (int kk = 0; kk < D / 16; ++kk) {
-                    const uint32_t off = (kk >> 2) * C::BOX_Q + (kk & 3) * 32;
-                    const uint64_t da = smem_desc_sw128(qa + off, 16, 1024);
-                    const uint64_t db = smem_desc_sw128(ka + off, 16, 1024);
-                    mma_ss(tmem + buf * BN, da, db, idS, kk > 0 ? 1u : 0u);
+                    const uint32_t off = (kk >> 2) * C::BOX + (kk & 3) * 32;
+                    mma_ss(tmem + C::s_col(t), smem_desc_sw128(qa + off, 16, 1024),
+                           smem_desc_sw128(ka + off, 16, 1024), idS, kk > 0 ? 1u : 0u);
                 }
-                mma_commit(bar(C::BAR_SFULL + buf));
+                mma_commit(bar(C::BAR_SFULL + t));
                 return true;
             };
-            auto issue_pv = [&](int it) -> bool {
-                const int st = it % C::NS;
-                const int buf = it & 1;
-                if (!mbar_wait(bar(C::BAR_PFULL + buf), (it >> 1) & 1, abort_flag, p.wait_limit_ns))
+            auto issue_pv = [&](int t, int u) -> bool {
+                const int g = u - u_lo;
+                const int st = g % C::NS;
+                const int i = u - TILE_LO(t);  // this tile's iteration index
+                if (!mbar_wait(bar(C::BAR_PFULL + t), i & 1, abort_flag, p.wait_limit_ns))
                     return false;
-                if (!mbar_wait(bar(C::BAR_VFULL + st), (it / C::NS) & 1, abort_flag,
+                if (!mbar_wait(bar(C::BAR_VFULL + st), (g / C::NS) & 1, abort_flag,
                                p.wait_limit_ns))
                     return false;
                 tc_fence_after();
                 const uint32_t va = sbase + C::OFF_V + st * C::KV_BYTES;
 #pragma unroll
-                for (int kk = 0; kk < BN / 16; ++kk) {
-                    const uint64_t db = smem_desc_sw128(va + kk * 16 * 128, C::BOX_KV, 1024);
-                    mma_ts(tmem + C::O_COL, tmem + buf * BN + kk * 8, db, idO,
-                           (it > 0 || kk > 0) ? 1u : 0u);
-                }
-                mma_commit(bar(C::BAR_EMPTY + st));
-                mma_commit(bar(C::BAR_ODONE));
+                for (int kk = 0; kk < BN / 16; ++kk)
+                    mma_ts(tmem + C::o_col(t), tmem + C::s_col(t) + kk * 8,
+                           smem_desc_sw128(va + kk * 16 * 128, C::BOX, 1024), idO,
+                           (i > 0 || kk > 0) ? 1u : 0u);
+                mma_commit(bar(C::BAR_ODONE + t));
                 return true;
             };
-            if (mbar_wait(bar(C::BAR_Q), 0, abort_flag, p.wait_limit_ns) && issue_s(0)) {
-                for (int it = 0; it < n_tiles; ++it) {
-                    if (it + 1 < n_tiles && !issue_s(it + 1)) break;
-                    if (!issue_pv(it)) break;
+            bool ok = mbar_wait(bar(C::BAR_Q), 0, abort_flag, p.wait_limit_ns);
+#pragma unroll
+            for (int t = 0; t < kTiles; ++t)
+                if (ok && USES(t, u_lo)) ok = issue_s(t, u_lo);
+            for (int u = u_lo; ok && u < u_hi; ++u) {
+#pragma unroll
+                for (int t = 0; t < kTiles; ++t) {
+                    if (ok && USES(t, u)) ok = issue_pv(t, u);
+                    if (ok && u + 1 < u_hi && USES(t, u + 1)) ok = issue_s(t, u + 1);
                 }
+                if (ok) mma_commit(bar(C::BAR_EMPTY + (u - u_lo) % C::NS));
             }
         }
-    } else if (warp < 4) {
+      }
+    } else {
         // ===================== softmax / correction / epilogue =====================
-        const int r = threadIdx.x;             // query row within the tile = TMEM lane
-        const int row = q0 + r;                // query row within the sequence
-        const uint32_t trow = tmem + (static_cast<uint32_t>(warp * 32) << 16);
+        regs_inc<kSoftmaxRegs>();
+        const int t = warp >> 2;                 // query tile of this warpgroup
+        const int r = threadIdx.x & (BM - 1);    // row within the tile = TMEM lane
+        const int row = (pair * kTiles + t) * BM + r;
+        const int q0 = (pair * kTiles + t) * BM;
+        const uint32_t trow = tmem + (static_cast<uint32_t>((warp & 3) * 32) << 16);
+        const uint32_t s_addr = trow + (t ? C::s_col(1) : C::s_col(0));
+        const uint32_t o_addr = trow + (t ? C::o_col(1) : C::o_col(0));
         const long long pos = (long long)p.input_pos + row;  // absolute position
-        float m_used = neg_inf();              // max subtracted so far (log2 units)
+        // this tile's range, selected without runtime-indexed arrays
+        const int my_lo = TILE_LO(t);
+        const int my_hi = TILE_HI(t);
+        const int my_qlast = t ? ql1 : ql0;
+        const int n_t = my_hi > my_lo ? my_hi - my_lo : 0;
+        const uint32_t bar_s = bar(C::BAR_SFULL + t), bar_p = bar(C::BAR_PFULL + t),
+                       bar_o = bar(C::BAR_ODONE + t);
+        float m_used = neg_inf();  // max subtracted so far (log2 units)
         float l = 0.f;
         bool ok = true;
 
-        for (int it = 0; it < n_tiles; ++it) {
-            const int buf = it & 1;
-            const int kv0 = (t_begin + it) * BN;
-            if (!warp_wait(bar(C::BAR_SFULL + buf), (it >> 1) & 1, abort_flag, p.wait_limit_ns)) {
+        for (int i = 0; i < n_t; ++i) {
+            const int u = my_lo + i;
+            const int g = u - u_lo;
+            const int kv0 = u * BN;
+            if (!warp_wait(bar_s, i & 1, abort_flag, p.wait_limit_ns)) {
                 ok = false;
                 break;
             }
             tc_fence_after();
-            float s[BN];
+            uint32_t sr[4][32];
 #pragma unroll
-            for (int c = 0; c < BN / 32; ++c) {
-                uint32_t v[32];
-                tmem_ld32(trow + buf * BN + c * 32, v);
-                tmem_wait_ld();
+            for (int c = 0; c < 4; ++c) tmem_ld32(s_addr + c * 32, sr[c]);
+            tmem_wait_ld();
 #pragma unroll
-                for (int k = 0; k < 32; ++k) s[c * 32 + k] = __uint_as_float(v[k]);
-            }
+            for (int c = 0; c < 4; ++c) reg_fence32(sr[c]);
+            float *s = reinterpret_cast<float *>(&sr[0][0]);
             // step a5: per-element mask on boundary tiles only
             const bool edge = (kv0 + BN > k_end) ||
                               (p.causal && (long long)kv0 + BN - 1 > (long long)p.input_pos + q0) ||
                               (p.window > 0 &&
-                               (long long)kv0 <= (long long)p.input_pos + q_last - p.window);
+                               (long long)kv0 <= (long long)p.input_pos + my_qlast - p.window);
             if (edge) {
                 long long hi = k_end;
                 if (p.causal) hi = min(hi, pos + 1);
-                long long lo = p.window > 0 ? pos - p.window + 1 : 0;
+                const long long lo = p.window > 0 ? pos - p.window + 1 : 0;
                 const int c_hi = static_cast<int>(max(-1ll, min((long long)BN, hi - kv0)));
                 const int c_lo = static_cast<int>(max(-1ll, min((long long)BN, lo - kv0)));
 #pragma unroll
                 for (int c = 0; c < BN; ++c) s[c] = (c >= c_lo && c < c_hi) ? s[c] : neg_inf();
             }
-            // step a6: online softmax in the exp2 domain, lazy rescaling
-            float mx = s[0];
+            // step a6: online softmax in the exp2 domain with lazy rescaling
+            float mx0 = s[0], mx1 = s[1];
 #pragma unroll
-            for (int c = 1; c < BN; ++c) mx = fmaxf(mx, s[c]);
-            const float m_new = mx * p.scale_log2;
+            for (int c = 2; c < BN; c += 2) {
+                mx0 = fmaxf(mx0, s[c]);
+                mx1 = fmaxf(mx1, s[c + 1]);
+            }
+            const float m_new = fmaxf(mx0, mx1) * p.scale_log2;
             float alpha = 1.f;
             bool resc = false;
             if (m_new > m_used + 8.f) {
@@ -284,73 +337,70 @@ __global__ void __launch_bounds__(kThreads, 1)
                 m_used = m_new;
                 resc = true;
             }
-            const float m_eff = (m_used == neg_inf()) ? 0.f : m_used;
-            float sum = 0.f;
-            uint32_t pk[BN / 2];
+            const float neg_m = (m_used == neg_inf()) ? 0.f : -m_used;
+            float sum0 = 0.f, sum1 = 0.f;
 #pragma unroll
-            for (int c = 0; c < BN / 2; ++c) {
-                const float p0 = fast_exp2(fmaf(s[2 * c], p.scale_log2, -m_eff));
-                const float p1 = fast_exp2(fmaf(s[2 * c + 1], p.scale_log2, -m_eff));
-                sum += p0 + p1;
-                pk[c] = pack_bf16x2(p0, p1);
+            for (int c = 0; c < 4; ++c) {
+                uint32_t pk[16];
+#pragma unroll
+                for (int k = 0; k < 16; ++k) {
+                    const float p0 = fast_exp2(fmaf(s[c * 32 + 2 * k], p.scale_log2, neg_m));
+                    const float p1 = fast_exp2(fmaf(s[c * 32 + 2 * k + 1], p.scale_log2, neg_m));
+                    sum0 += p0;
+                    sum1 += p1;
+                    pk[k] = pack_bf16x2(p0, p1);
+                }
+                tmem_st16(s_addr + c * 16, pk);
             }
-            l = l * alpha + sum;
+            l = l * alpha + (sum0 + sum1);
+            // O correction.  S_t(i) completing implies P_t(i-1) V has completed (same
+            // issuing thread, in order), so O_t is quiet until we arrive on P_FULL.
+            if (i > 0 && __any_sync(0xffffffffu, resc)) {
 #pragma unroll
-            for (int c = 0; c < BN / 64; ++c) {
-                uint32_t v[32];
+                for (int c = 0; c < D / 32; ++c) {
+                    uint32_t v[32];
+                    tmem_ld32(o_addr + c * 32, v);
+                    tmem_wait_ld();
+                    reg_fence32(v);
 #pragma unroll
-                for (int k = 0; k < 32; ++k) v[k] = pk[c * 32 + k];
-                tmem_st32(trow + buf * BN + c * 32, v);
+                    for (int k = 0; k < 32; ++k)
+                        v[k] = __float_as_uint(__uint_as_float(v[k]) * alpha);
+                    tmem_st32(o_addr + c * 32, v);
+                }
             }
             // Key rows at or past k_end inside this tile may hold anything; their
-            // weights are exactly 0, but 0 * NaN is NaN, so zero those V rows.
-            if (k_end < p.Sk && k_end > kv0 && k_end < kv0 + BN) {
-                const int st = it % C::NS;
-                if (!warp_wait(bar(C::BAR_VFULL + st), (it / C::NS) & 1, abort_flag,
+            // weights are exactly 0, but 0 * NaN is NaN, so zero those V rows (done
+            // by the first query tile that uses this KV tile).
+            if (k_end < p.Sk && k_end > kv0 && k_end < kv0 + BN && (t == 0 || !USES(0, u))) {
+                const int st = g % C::NS;
+                if (!warp_wait(bar(C::BAR_VFULL + st), (g / C::NS) & 1, abort_flag,
                                p.wait_limit_ns)) {
                     ok = false;
-                }
-                if (ok && r >= k_end - kv0 && r < p.Sk - kv0) {
-#pragma unroll
-                    for (int c = 0; c < C::NBOX; ++c) {
-                        uint4 *dst = reinterpret_cast<uint4 *>(smem + C::OFF_V + st * C::KV_BYTES +
-                                                               c * C::BOX_KV + r * 128);
-#pragma unroll
-                        for (int k = 0; k < 8; ++k) dst[k] = make_uint4(0, 0, 0, 0);
-                    }
-                }
-                fence_proxy_async_smem();
-                __syncwarp();
-            }
-            // O correction: only when some row of this warp moved its max by > 8
-            if (ok && it > 0 && __any_sync(0xffffffffu, resc)) {
-                if (!warp_wait(bar(C::BAR_ODONE), (it - 1) & 1, abort_flag, p.wait_limit_ns)) {
-                    ok = false;
                 } else {
-                    tc_fence_after();
+                    if (r >= k_end - kv0 && r < p.Sk - kv0) {
 #pragma unroll
-                    for (int c = 0; c < D / 32; ++c) {
-                        uint32_t v[32];
-                        tmem_ld32(trow + C::O_COL + c * 32, v);
-                        tmem_wait_ld();
+                        for (int c = 0; c < C::NBOX; ++c) {
+                            uint4 *dst = reinterpret_cast<uint4 *>(
+                                smem + C::OFF_V + st * C::KV_BYTES + c * C::BOX + r * 128);
 #pragma unroll
-                        for (int k = 0; k < 32; ++k)
-                            v[k] = __float_as_uint(__uint_as_float(v[k]) * alpha);
-                        tmem_st32(trow + C::O_COL + c * 32, v);
+                            for (int k = 0; k < 8; ++k) dst[k] = make_uint4(0, 0, 0, 0);
+                        }
                     }
+                    fence_proxy_async_smem();
                 }
+                __syncwarp();
             }
             tmem_wait_st();
             tc_fence_before();
-            mbar_arrive(bar(C::BAR_PFULL + buf));
+            mbar_arrive(bar_p);
             if (!ok) break;
         }
 
         // step a8: epilogue
         const bool row_in = row < p.Sq;
-        bool have = ok && n_tiles > 0;
+        bool have = ok && n_t > 0;
         if (have &&
-            !warp_wait(bar(C::BAR_ODONE), (n_tiles - 1) & 1, abort_flag, p.wait_limit_ns))
+            !warp_wait(bar_o, (n_t - 1) & 1, abort_flag, p.wait_limit_ns))
             have = false;
         const bool out_valid = have && row < q_end && l > 0.f;
         const float inv_l = out_valid ? 1.f / l : 0.f;
@@ -360,8 +410,9 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
             for (int c = 0; c < D / 32; ++c) {
                 uint32_t v[32];
-                tmem_ld32(trow + C::O_COL + c * 32, v);
+                tmem_ld32(o_addr + c * 32, v);
                 tmem_wait_ld();
+                reg_fence32(v);
                 uint32_t o16[16];
 #pragma unroll
                 for (int k = 0; k < 16; ++k)
@@ -386,11 +437,14 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
     }
 
+#undef TILE_LO
+#undef TILE_HI
+#undef USES
     // ---- teardown ----
     if (*abort_flag) drain_delay(2000000);  // let copies / MMAs in flight land
     tc_fence_before();
     __syncthreads();
-    if (warp == 5) {
+    if (warp == kWarpMma) {
         __syncwarp();
         tc_fence_after();
         tmem_dealloc(tmem, C::TMEM_COLS);
@@ -407,6 +461,12 @@ attn_status_t launch_fwd_d(const FwdArgs &a, cudaStream_t stream) {
     if ((st = make_tmap_bf16_3d(&tv, a.V, D, a.Sk, (uint64_t)a.B * a.Hkv, BN)) != ATTN_OK) return st;
     static bool configured = false;
     if (!configured) {
+        // The register hand-over inside the kernel assumes exactly kLaunchRegs
+        // registers per thread at launch; refuse to launch a build where it differs.
+        cudaFuncAttributes fa;
+        if (cudaFuncGetAttributes(&fa, attn_fwd_kernel<D>) != cudaSuccess ||
+            fa.numRegs != kLaunchRegs)
+            return ATTN_ERR_CUDA;
         if (cudaFuncSetAttribute(attn_fwd_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                  C::SMEM_BYTES) != cudaSuccess)
             return ATTN_ERR_CUDA;
@@ -423,13 +483,13 @@ attn_status_t launch_fwd_d(const FwdArgs &a, cudaStream_t stream) {
     p.Sq = a.Sq;
     p.Sk = a.Sk;
     p.group = a.Hq / a.Hkv;
-    p.n_qtiles = (a.Sq + BM - 1) / BM;
+    p.n_pairs = (a.Sq + kTiles * BM - 1) / (kTiles * BM);
     p.scale_log2 = a.scale * 1.4426950408889634f;
     p.causal = a.causal;
     p.window = a.window;
     p.input_pos = a.input_pos;
     p.wait_limit_ns = kWaitLimitNs;
-    const long long grid = (long long)p.n_qtiles * a.Hq * a.B;
+    const long long grid = (long long)p.n_pairs * a.Hq * a.B;
     if (grid == 0) return ATTN_OK;
     if (grid > 0x7fffffffll) return ATTN_ERR_INVALID;
     attn_fwd_kernel<D><<<static_cast<unsigned>(grid), kThreads, C::SMEM_BYTES, stream>>>(tq, tk, tv,
