@@ -42,7 +42,7 @@ def up_to_date(output: str = LIBRARY) -> bool:
 def build(output: str = LIBRARY, verbose_ptxas: bool = False, force: bool = False) -> str:
     if not force and up_to_date(output):
         return output
-    cmd = [nvcc(), *ARCH, "-O3", "-lineinfo", "-std=c++17", "-rdc=true", "-shared",
+    cmd = [nvcc(), *ARCH, "-O3", "-lineinfo", "-std=c++17", "-shared",
            "-Xcompiler", "-fPIC", "-I", INCLUDE, "-I", CSRC, *sources(), "-o", output]
     if verbose_ptxas:
         cmd[1:1] = ["-Xptxas", "-v"]

@@ -16,6 +16,23 @@ namespace gqa {
 
 __device__ int g_status = 0;
 
+namespace {
+std::mutex g_status_mutex;
+int *g_status_ptr[64] = {};
+}  // namespace
+
+int *device_status_word() {
+    int dev = -1;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return nullptr;
+    std::lock_guard<std::mutex> lock(g_status_mutex);
+    if (g_status_ptr[dev] == nullptr) {
+        void *ptr = nullptr;
+        if (cudaGetSymbolAddress(&ptr, g_status) != cudaSuccess) return nullptr;
+        g_status_ptr[dev] = static_cast<int *>(ptr);
+    }
+    return g_status_ptr[dev];
+}
+
 size_t decode_workspace_floats(int B, int Hq, int n_splits, int D);
 
 namespace {
@@ -70,7 +87,7 @@ __global__ void wait_probe_kernel(uint64_t limit_ns) {
     }
     __syncthreads();
     // Nobody arrives on `bar`: the bounded wait must give up and record the status.
-    warp_wait(b, 0, &abort_flag, limit_ns);
+    warp_wait(b, 0, &abort_flag, limit_ns, &g_status);
     __syncthreads();
 }
 

@@ -59,6 +59,7 @@ struct DecParams {
     int B, Hq, Hkv, S_cap, group, n_splits;
     float scale_log2;
     uint64_t wait_limit_ns;
+    int *status;  // device status word
 };
 
 __device__ __forceinline__ float neg_inf() { return __int_as_float(0xff800000); }
@@ -92,7 +93,7 @@ __global__ void __launch_bounds__(kDecThreads)
 
     int len = p.lengths[b];
     if (len > p.S_cap) {
-        if (threadIdx.x == 0 && split == 0 && hkv == 0) record_status(ATTN_ERR_DEVICE_BOUNDS);
+        if (threadIdx.x == 0 && split == 0 && hkv == 0) record_status(p.status, ATTN_ERR_DEVICE_BOUNDS);
         len = p.S_cap;
     }
     if (len < 0) len = 0;
@@ -130,7 +131,7 @@ __global__ void __launch_bounds__(kDecThreads)
                 const int st = it % C::NS;
                 const int use = it / C::NS;
                 if (use > 0 &&
-                    !mbar_wait(empty(st), (use - 1) & 1, abort_flag, p.wait_limit_ns))
+                    !mbar_wait(empty(st), (use - 1) & 1, abort_flag, p.wait_limit_ns, p.status))
                     break;
                 const int row = (t_begin + it) * TN;
                 mbar_arrive_expect_tx(full(st), 2 * C::TILE);
@@ -172,7 +173,7 @@ __global__ void __launch_bounds__(kDecThreads)
         bool ok = true;
         for (int it = 0; it < n_tiles; ++it) {
             const int st = it % C::NS;
-            if (!warp_wait(full(st), (it / C::NS) & 1, abort_flag, p.wait_limit_ns)) {
+            if (!warp_wait(full(st), (it / C::NS) & 1, abort_flag, p.wait_limit_ns, p.status)) {
                 ok = false;
                 break;
             }
@@ -385,6 +386,8 @@ attn_status_t launch_decode_d(const DecodeArgs &a, cudaStream_t stream) {
     p.n_splits = a.n_splits;
     p.scale_log2 = 1.4426950408889634f / sqrtf(static_cast<float>(D));
     p.wait_limit_ns = kWaitLimitNs;
+    p.status = device_status_word();
+    if (!p.status) return ATTN_ERR_CUDA;
     dim3 grid(a.n_splits, a.Hkv, a.B);
     decode_split_kernel<D><<<grid, kDecThreads, C::SMEM_BYTES, stream>>>(tk, tv, p);
     if (cudaGetLastError() != cudaSuccess) return ATTN_ERR_CUDA;

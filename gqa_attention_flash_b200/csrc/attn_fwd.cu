@@ -18,8 +18,9 @@
 //              from TMEM, written there by the softmax over S_t)
 //   warps 10-11 idle
 // The block launches with 168 registers per thread; the producer warpgroup
-// (warps 8-11) drops to 56 and the two softmax warpgroups rise to 224
-// (128 * 56 + 256 * 224 = 384 * 168).
+// (warps 8-11) drops to 64 and the two softmax warpgroups rise to 216
+// (128 * 64 + 256 * 216 <= 384 * 168).  Every translation unit is compiled as a
+// whole program: with relocatable device code ptxas would ignore setmaxnreg.
 // TMEM (512 columns): S0 | S1 | O0 | O1.  Each query tile visits only the KV
 // tiles that hold a key it can see (whole-tile skipping for causal, window and
 // length masks -- Tylo `flex_attention!` keyword block_sparse); the
@@ -40,8 +41,8 @@ constexpr int kWarpTma = 8;
 constexpr int kWarpMma = 9;
 constexpr int kThreads = 384;
 constexpr int kLaunchRegs = 168;     // per thread at launch (checked on the host)
-constexpr uint32_t kProducerRegs = 56;
-constexpr uint32_t kSoftmaxRegs = 224;
+constexpr uint32_t kProducerRegs = 64;
+constexpr uint32_t kSoftmaxRegs = 216;
 static_assert(128 * kProducerRegs + 256 * kSoftmaxRegs <= kThreads * kLaunchRegs,
               "register split must use exactly the launch allocation");
 
@@ -80,6 +81,7 @@ struct FwdParams {
     float scale_log2;  // scale * log2(e)
     int causal, window, input_pos;
     uint64_t wait_limit_ns;
+    int *status;  // device status word
 };
 
 __device__ __forceinline__ float neg_inf() { return __int_as_float(0xff800000); }
@@ -114,7 +116,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (p.k_lengths) {
         int kl = p.k_lengths[b];
         if (kl > p.Sk) {
-            if (threadIdx.x == 0 && hq == 0 && pair == 0) record_status(ATTN_ERR_DEVICE_BOUNDS);
+            if (threadIdx.x == 0 && hq == 0 && pair == 0) record_status(p.status, ATTN_ERR_DEVICE_BOUNDS);
             kl = p.Sk;
         }
         k_end = kl > 0 ? kl : 0;
@@ -122,7 +124,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (p.q_lengths) {
         int ql = p.q_lengths[b];
         if (ql > p.Sq) {
-            if (threadIdx.x == 0 && hq == 0 && pair == 0) record_status(ATTN_ERR_DEVICE_BOUNDS);
+            if (threadIdx.x == 0 && hq == 0 && pair == 0) record_status(p.status, ATTN_ERR_DEVICE_BOUNDS);
             ql = p.Sq;
         }
         q_end = ql > 0 ? ql : 0;
@@ -201,7 +203,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 const int st = g % C::NS;
                 const int use = g / C::NS;
                 if (use > 0 &&
-                    !mbar_wait(bar(C::BAR_EMPTY + st), (use - 1) & 1, abort_flag, p.wait_limit_ns))
+                    !mbar_wait(bar(C::BAR_EMPTY + st), (use - 1) & 1, abort_flag, p.wait_limit_ns, p.status))
                     break;
                 const int kv_row = (u_lo + g) * BN;
                 mbar_arrive_expect_tx(bar(C::BAR_KFULL + st), C::KV_BYTES);
@@ -223,7 +225,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 const int g = u - u_lo;
                 const int st = g % C::NS;
                 if (!mbar_wait(bar(C::BAR_KFULL + st), (g / C::NS) & 1, abort_flag,
-                               p.wait_limit_ns))
+                               p.wait_limit_ns, p.status))
                     return false;
                 tc_fence_after();
                 const uint32_t qa = sbase + C::OFF_Q + t * C::Q_BYTES;
@@ -241,10 +243,10 @@ __global__ void __launch_bounds__(kThreads, 1)
                 const int g = u - u_lo;
                 const int st = g % C::NS;
                 const int i = u - TILE_LO(t);  // this tile's iteration index
-                if (!mbar_wait(bar(C::BAR_PFULL + t), i & 1, abort_flag, p.wait_limit_ns))
+                if (!mbar_wait(bar(C::BAR_PFULL + t), i & 1, abort_flag, p.wait_limit_ns, p.status))
                     return false;
                 if (!mbar_wait(bar(C::BAR_VFULL + st), (g / C::NS) & 1, abort_flag,
-                               p.wait_limit_ns))
+                               p.wait_limit_ns, p.status))
                     return false;
                 tc_fence_after();
                 const uint32_t va = sbase + C::OFF_V + st * C::KV_BYTES;
@@ -256,7 +258,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 mma_commit(bar(C::BAR_ODONE + t));
                 return true;
             };
-            bool ok = mbar_wait(bar(C::BAR_Q), 0, abort_flag, p.wait_limit_ns);
+            bool ok = mbar_wait(bar(C::BAR_Q), 0, abort_flag, p.wait_limit_ns, p.status);
 #pragma unroll
             for (int t = 0; t < kTiles; ++t)
                 if (ok && USES(t, u_lo)) ok = issue_s(t, u_lo);
@@ -296,7 +298,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             const int u = my_lo + i;
             const int g = u - u_lo;
             const int kv0 = u * BN;
-            if (!warp_wait(bar_s, i & 1, abort_flag, p.wait_limit_ns)) {
+            if (!warp_wait(bar_s, i & 1, abort_flag, p.wait_limit_ns, p.status)) {
                 ok = false;
                 break;
             }
@@ -374,7 +376,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             if (k_end < p.Sk && k_end > kv0 && k_end < kv0 + BN && (t == 0 || !USES(0, u))) {
                 const int st = g % C::NS;
                 if (!warp_wait(bar(C::BAR_VFULL + st), (g / C::NS) & 1, abort_flag,
-                               p.wait_limit_ns)) {
+                               p.wait_limit_ns, p.status)) {
                     ok = false;
                 } else {
                     if (r >= k_end - kv0 && r < p.Sk - kv0) {
@@ -400,7 +402,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         const bool row_in = row < p.Sq;
         bool have = ok && n_t > 0;
         if (have &&
-            !warp_wait(bar_o, (n_t - 1) & 1, abort_flag, p.wait_limit_ns))
+            !warp_wait(bar_o, (n_t - 1) & 1, abort_flag, p.wait_limit_ns, p.status))
             have = false;
         const bool out_valid = have && row < q_end && l > 0.f;
         const float inv_l = out_valid ? 1.f / l : 0.f;
@@ -489,6 +491,8 @@ attn_status_t launch_fwd_d(const FwdArgs &a, cudaStream_t stream) {
     p.window = a.window;
     p.input_pos = a.input_pos;
     p.wait_limit_ns = kWaitLimitNs;
+    p.status = device_status_word();
+    if (!p.status) return ATTN_ERR_CUDA;
     const long long grid = (long long)p.n_pairs * a.Hq * a.B;
     if (grid == 0) return ATTN_OK;
     if (grid > 0x7fffffffll) return ATTN_ERR_INVALID;

@@ -33,6 +33,10 @@ struct DecodeArgs {
     float *workspace;  // B * Hq * n_splits * (D + 1) floats
 };
 
+// Device address of the status word on the current device (looked up once per
+// device), or nullptr if the lookup failed.
+int *device_status_word();
+
 attn_status_t launch_fwd(const FwdArgs &a, cudaStream_t stream);
 attn_status_t launch_decode(const DecodeArgs &a, cudaStream_t stream);
 attn_status_t launch_wait_probe(int limit_us, cudaStream_t stream);

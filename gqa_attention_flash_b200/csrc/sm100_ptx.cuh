@@ -12,11 +12,11 @@
 
 namespace gqa {
 
-// Per-device status word; kernels record the first error they meet.
-extern __device__ int g_status;
-
-__device__ __forceinline__ void record_status(int code) {
-    atomicCAS(&g_status, 0, code);
+// Kernels record the first error they meet in a per-device status word whose
+// device address the host passes in (so every translation unit stays
+// self-contained and is compiled as a whole program).
+__device__ __forceinline__ void record_status(int *status, int code) {
+    if (status) atomicCAS(status, 0, code);
 }
 
 __device__ __forceinline__ uint32_t smem_u32(const void *p) {
@@ -67,7 +67,7 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
 // ATTN_ERR_TIMEOUT and returns false.  Every caller treats false as "stop
 // issuing work and head for the exit path".
 __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatile int *abort_flag,
-                                          uint64_t limit_ns) {
+                                          uint64_t limit_ns, int *status) {
     if (mbar_try_wait(bar, parity)) return true;
     const uint64_t t0 = global_timer_ns();
     for (uint32_t it = 1;; ++it) {
@@ -76,7 +76,7 @@ __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatil
             if (*abort_flag) return false;
             if (global_timer_ns() - t0 > limit_ns) {
                 *abort_flag = 1;
-                record_status(ATTN_ERR_TIMEOUT);
+                record_status(status, ATTN_ERR_TIMEOUT);
                 return false;
             }
         }
@@ -87,8 +87,8 @@ __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatil
 // all lanes saw the phase complete.  Keeps later warp-collective instructions
 // (tcgen05.ld/st, vote) converged on the give-up path.
 __device__ __forceinline__ bool warp_wait(uint32_t bar, uint32_t parity, volatile int *abort_flag,
-                                          uint64_t limit_ns) {
-    const bool w = mbar_wait(bar, parity, abort_flag, limit_ns);
+                                          uint64_t limit_ns, int *status) {
+    const bool w = mbar_wait(bar, parity, abort_flag, limit_ns, status);
     return __all_sync(0xffffffffu, w);
 }
 

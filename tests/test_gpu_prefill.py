@@ -100,3 +100,24 @@ def test_full_size_sampled(orc, name):
     Or, Lr = oracle_prefill(orc, x.Q, x.K, x.V, w.scale, w.causal, w.window, w.input_pos,
                             x.k_lengths, x.q_lengths, rows=rows)
     compare(O, L, Or, Lr, rows=rows, what=name)
+
+
+@pytest.mark.parametrize("causal", [False, True])
+def test_running_max_jumps(orc, causal):
+    """Keys with scores far above the rest appear deep into the rows (different KV
+    tiles for different rows), so the running row max jumps by more than 2^8 after
+    a row's first tile: this exercises the redo of a tile's exponentials and the
+    rescaling of the O accumulator."""
+    B, Hq, Hkv, S, D = 1, 4, 2, 1100, 128
+    Q, K, V = W.random_prefill(21, B, Hq, Hkv, S, S, D)
+    K = K.float()
+    for j, f in [(300, 8.0), (700, 14.0), (1030, 20.0)]:
+        K[:, :, j] *= f
+    K = K.to(torch.bfloat16)
+    # such rows return nearly one V row; keep |V| < 2 so that bf16 rounding of O
+    # (2^-7 there) stays well inside the tolerance
+    V = (V.float() * 0.5).clamp(-1.9, 1.9).to(torch.bfloat16)
+    scale = 1.0 / np.sqrt(D)
+    O, L = gpu_prefill(Q, K, V, scale, causal)
+    Or, Lr = oracle_prefill(orc, Q, K, V, scale, causal)
+    compare(O, L, Or, Lr, what=f"max jumps causal={causal}")
