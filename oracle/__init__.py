@@ -68,6 +68,10 @@ class Oracle:
         L.oracle_attn_fwd.restype = ctypes.c_int
         L.oracle_attn_fwd.argtypes = [_D, _D, _D, _D, _D] + [ctypes.c_int] * 6 + [
             ctypes.c_double, ctypes.c_int, ctypes.c_int, ctypes.c_int, _I, _I, _I, ctypes.c_int]
+        L.oracle_flex_fwd.restype = ctypes.c_int
+        L.oracle_flex_fwd.argtypes = [_D, _D, _D, _D, _D] + [ctypes.c_int] * 6 + [
+            ctypes.c_double, ctypes.c_int, ctypes.c_int, ctypes.c_int, _I, _I, _I, ctypes.c_int,
+            ctypes.c_double, _D, _I, _I]
         L.oracle_decode.restype = ctypes.c_int
         L.oracle_decode.argtypes = [_D, _D, _D, _D, _D] + [ctypes.c_int] * 5 + [_I]
 
@@ -113,6 +117,42 @@ class Oracle:
                                       _iptr(rows_a), n)
         if rc != 0:
             raise ValueError("oracle_attn_fwd rejected its arguments")
+        return O, LSE
+
+    # -- Tylo.jl "Primitives" page, flex_attention! -----------------------------------
+    def flex_fwd(self, Q, K, V, scale, causal=False, window=0, input_pos=0,
+                 k_lengths=None, q_lengths=None, rows=None, Sq=None,
+                 softcap=0.0, alibi_slopes=None, doc_q=None, doc_kv=None):
+        """attn_fwd with SoftCapScore / AliBiScore and DocumentMask.
+
+        ``doc_q`` has one id per local query row (length Sq), ``doc_kv`` one per
+        key (length Sk); ``alibi_slopes`` one slope per query head.
+        """
+        Q, K, V = _f64(Q), _f64(K), _f64(V)
+        B, Hq, n, D = Q.shape
+        Bk, Hkv, Sk, Dk = K.shape
+        assert Bk == B and Dk == D and V.shape == K.shape
+        rows_a = _i32(rows)
+        if rows_a is None:
+            Sq = n
+        else:
+            assert rows_a.shape == (n,) and Sq is not None
+        kl, ql = _i32(k_lengths), _i32(q_lengths)
+        sl = None if alibi_slopes is None else _f64(alibi_slopes)
+        if sl is not None:
+            assert sl.shape == (Hq,)
+        dq, dk = _i32(doc_q), _i32(doc_kv)
+        if dq is not None:
+            assert dq.shape == (Sq,) and dk is not None and dk.shape == (Sk,)
+        O = np.empty((B, Hq, n, D), dtype=np.float64)
+        LSE = np.empty((B, Hq, n), dtype=np.float64)
+        rc = self.lib.oracle_flex_fwd(_dptr(O), _dptr(LSE), _dptr(Q), _dptr(K), _dptr(V),
+                                      B, Hq, Hkv, Sq, Sk, D, float(scale), int(causal),
+                                      int(window), int(input_pos), _iptr(kl), _iptr(ql),
+                                      _iptr(rows_a), n, float(softcap), _dptr(sl),
+                                      _iptr(dq), _iptr(dk))
+        if rc != 0:
+            raise ValueError("oracle_flex_fwd rejected its arguments")
         return O, LSE
 
     # -- Tylo.jl "Primitives" page, decode_attention! ---------------------------------

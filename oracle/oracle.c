@@ -22,6 +22,14 @@
  *   - Tylo.jl "Primitives" page, entry `CausalMask`: a query sees keys at or
  *     before its own position, positions being absolute (input_pos shifts the
  *     queries).
+ *   - Tylo.jl "Primitives" page, entry `flex_attention!` with the score mods
+ *     `SoftCapScore(cap)` (s -> cap * tanh(s / cap)) and `AliBiScore(slopes)`
+ *     (adds slopes[h] * (q - kv), absolute positions) and the mask mod
+ *     `DocumentMask(doc_q, doc_kv)` (a pair attends iff the document ids of
+ *     the query and the key match), combined with the masks above.  The
+ *     precomputed `BlockMask` only tells a kernel which tiles to skip; when it
+ *     agrees with the mask mod (as the page requires) it changes nothing in
+ *     the result, so the oracle ignores it.
  *   - Tylo.jl "Primitives" page, entry `decode_attention!`: one query vector
  *     per head and sequence against the first lengths[b] cached keys.  The
  *     split into n_splits slices and their combine change only the rounding,
@@ -37,6 +45,14 @@
  *     position p iff p - w < j <= p, i.e. at most w keys, itself included.
  *   - a row with no visible key (invalid row, empty length, or every key cut)
  *     has O = 0 and LSE = -inf.
+ *   - score mods act on the scaled score s = scale * <q, k>; at most one of
+ *     them per call (the page composes mods with ComposeScore, whose order a
+ *     caller would fix; no such composition is built).  The ALiBi distance
+ *     is (input_pos + i) - j, the absolute query position minus the key
+ *     position, with the sign the page gives.
+ *   - document ids: doc_q[i] belongs to local query row i (absolute position
+ *     input_pos + i), doc_kv[j] to key j; both are shared by every batch
+ *     entry and head.
  *
  * Precision: inputs are doubles (the harness widens the exact bf16 values),
  * every product, sum, exp and log is done in double.
@@ -182,6 +198,99 @@ int oracle_attn_fwd(double *O, double *LSE, const double *Q, const double *K, co
                 for (int d = 0; d < D; ++d) o[d] += p * Vb[j * D + d];
             }
             if (LSE) LSE[(b * Hq + hq) * (long)n_rows + r] = mx + log(l);
+        }
+        free(score);
+        free(mask);
+    }
+    return bad ? -1 : 0;
+}
+
+/*
+ * Tylo.jl "Primitives" page, `flex_attention!`: the `attention!` rows above
+ * with a score mod and a document mask.  For each requested row, every key j:
+ *   s_j = scale * <Q_i, K_j>
+ *   if softcap > 0:        s_j = softcap * tanh(s_j / softcap)   (SoftCapScore)
+ *   else if alibi_slopes:  s_j += alibi_slopes[hq] * ((input_pos + i) - j)
+ *                                                                (AliBiScore)
+ *   visible_j = the causal / window / length rule of mask_row, and, if doc_q
+ *               and doc_kv are given, doc_q[i] == doc_kv[j]       (DocumentMask)
+ *   then the softmax, O and LSE exactly as in oracle_attn_fwd.
+ * Returns 0, or -1 on bad arguments.
+ */
+int oracle_flex_fwd(double *O, double *LSE, const double *Q, const double *K, const double *V,
+                    int B, int Hq, int Hkv, int Sq, int Sk, int D, double scale,
+                    int causal, int window, int input_pos,
+                    const int *k_lengths, const int *q_lengths,
+                    const int *rows, int n_rows,
+                    double softcap, const double *alibi_slopes,
+                    const int *doc_q, const int *doc_kv) {
+    if (B < 0 || Hq <= 0 || Hkv <= 0 || Sq < 0 || Sk < 0 || D <= 0) return -1;
+    if (Hq % Hkv != 0) return -1;
+    if (window > 0 && !causal) return -1;
+    if (softcap < 0.0) return -1;
+    if (softcap > 0.0 && alibi_slopes != NULL) return -1; /* composition order not fixed */
+    if ((doc_q == NULL) != (doc_kv == NULL)) return -1;
+    if (rows == NULL) n_rows = Sq;
+    const int group = Hq / Hkv;
+    const long total = (long)B * Hq * n_rows;
+    int bad = 0;
+
+#pragma omp parallel
+    {
+        double *score = (double *)malloc(sizeof(double) * (Sk > 0 ? Sk : 1));
+        double *mask = (double *)malloc(sizeof(double) * (Sk > 0 ? Sk : 1));
+        if (score == NULL || mask == NULL) {
+#pragma omp atomic write
+            bad = 1;
+        }
+#pragma omp for schedule(dynamic, 16)
+        for (long t = 0; t < total; ++t) {
+            if (score == NULL || mask == NULL) continue;
+            const long r = t % n_rows;
+            const long hq = (t / n_rows) % Hq;
+            const long b = t / ((long)n_rows * Hq);
+            const long i = rows ? rows[r] : r;
+            const long kv_head = hq / group;
+            const long row_id = (b * Hq + hq) * (long)n_rows + r;
+            const int k_len = k_lengths ? k_lengths[b] : Sk;
+            const int q_len = q_lengths ? q_lengths[b] : Sq;
+            const double q_pos = (double)((long)input_pos + i);
+
+            const double *q = Q + row_id * D;
+            const double *Kb = K + (b * Hkv + kv_head) * (long)Sk * D;
+            const double *Vb = V + (b * Hkv + kv_head) * (long)Sk * D;
+            double *o = O + row_id * D;
+
+            mask_row(mask, i, Sk, causal, window, input_pos, k_len, q_len);
+            if (doc_q != NULL)
+                for (long j = 0; j < Sk; ++j)
+                    if (doc_q[i] != doc_kv[j]) mask[j] = -INFINITY;
+            double mx = -INFINITY;
+            for (long j = 0; j < Sk; ++j) {
+                double dot = 0.0;
+                for (int d = 0; d < D; ++d) dot += q[d] * Kb[j * D + d];
+                double sj = scale * dot;
+                if (softcap > 0.0) sj = softcap * tanh(sj / softcap);
+                if (alibi_slopes != NULL) sj += alibi_slopes[hq] * (q_pos - (double)j);
+                score[j] = sj + mask[j];
+                if (score[j] > mx) mx = score[j];
+            }
+            for (int d = 0; d < D; ++d) o[d] = 0.0;
+            if (mx == -INFINITY) {
+                if (LSE) LSE[row_id] = -INFINITY;
+                continue;
+            }
+            double lsum = 0.0;
+            for (long j = 0; j < Sk; ++j) {
+                score[j] = exp(score[j] - mx);
+                lsum += score[j];
+            }
+            for (long j = 0; j < Sk; ++j) {
+                const double pj = score[j] / lsum;
+                if (pj == 0.0) continue;
+                for (int d = 0; d < D; ++d) o[d] += pj * Vb[j * D + d];
+            }
+            if (LSE) LSE[row_id] = mx + log(lsum);
         }
         free(score);
         free(mask);

@@ -333,6 +333,95 @@ def pin_decode_closed_forms(orc):
     assert abs(L1[0, 0] - 1.0) < 1e-12, L1
 
 
+# --------------------------------------------------------------------------------------
+# Tylo.jl "Primitives" page: flex_attention! score and mask mods
+# --------------------------------------------------------------------------------------
+
+def pin_flex_golden(orc):
+    """Hand-derived soft-cap and ALiBi values in golden/flex_score_mods.json."""
+    with open(os.path.join(GOLDEN, "flex_score_mods.json")) as f:
+        g = json.load(f)
+    sc = g["softcap"]
+    q = np.array(sc["q"], dtype=np.float64)[None, None]
+    k = np.array(sc["k"], dtype=np.float64)[None, None]
+    v = np.array(sc["v"], dtype=np.float64)[None, None]
+    ln3 = math.log(3.0)
+    O, L = orc.flex_fwd(q, k, v, ln3 * ln3, softcap=2.0 * ln3)
+    assert abs(O[0, 0, 0, 0] - sc["O"][0]) < 1e-12, O
+    assert abs(L[0, 0, 0] - math.log(sc["LSE_is_ln"])) < 1e-12, L
+    al = g["alibi"]
+    Sk, row = al["Sk"], al["row"]
+    slopes = np.array(al["slopes_in_units_of_ln2"]) * math.log(2.0)
+    Q = np.zeros((1, 2, Sk, Sk))
+    K = np.zeros((1, 1, Sk, Sk))
+    V = np.eye(Sk)[None, None]
+    O, L = orc.flex_fwd(Q, K, V, 0.7, causal=True, alibi_slopes=slopes)
+    for h in range(2):
+        assert np.allclose(O[0, h, row], al["p"][h], rtol=0, atol=1e-12), (h, O[0, h, row])
+        assert abs(L[0, h, row] - math.log(al["LSE_is_ln"][h])) < 1e-12, (h, L[0, h, row])
+
+
+def pin_flex_softcap_limits(orc):
+    """A cap far above every score changes nothing (cap * tanh(s / cap) -> s): the
+    result equals attention! without a score mod.  A cap far below every score
+    flattens them to ~0: uniform weights over the visible keys, LSE = ln(count)."""
+    rng = _rng(21)
+    Q, K, V = rng.standard_normal((2, 4, 9, 8)), rng.standard_normal((2, 2, 11, 8)), \
+        rng.standard_normal((2, 2, 11, 8))
+    O0, L0 = orc.attn_fwd(Q, K, V, 0.4, causal=True, input_pos=2)
+    O1, L1 = orc.flex_fwd(Q, K, V, 0.4, causal=True, input_pos=2, softcap=1e9)
+    assert np.max(np.abs(O1 - O0)) < 1e-9 and np.max(np.abs(L1 - L0)) < 1e-9
+    O2, L2 = orc.flex_fwd(Q, K, V, 0.4, causal=True, input_pos=2, softcap=1e-12)
+    for i in range(9):
+        n = i + 3  # keys 0 .. input_pos + i
+        mean = V[:, :, :n].mean(axis=2)  # (B, Hkv, D)
+        assert np.allclose(O2[:, :, i], np.repeat(mean, 2, axis=1), rtol=0, atol=1e-9)
+        assert np.allclose(L2[:, :, i], math.log(n), rtol=0, atol=1e-9)
+
+
+def pin_flex_alibi_geometric(orc):
+    """With K = 0 the ALiBi scores are slope * (q - j): the weights over the visible
+    keys of a causal row are geometric, p_j = r^(q-j) / sum_k r^(q-k) with
+    r = exp(slope), and LSE = ln sum_k r^(q-k).  Checked per query head (GQA group
+    of 3 sharing one KV head, three different slopes) and with input_pos > 0."""
+    Sk, input_pos, Sq = 7, 3, 4
+    slopes = np.array([0.35, -0.6, 1.1])
+    Q = np.zeros((1, 3, Sq, Sk))
+    K = np.zeros((1, 1, Sk, Sk))
+    V = np.eye(Sk)[None, None]
+    O, L = orc.flex_fwd(Q, K, V, 1.3, causal=True, input_pos=input_pos, alibi_slopes=slopes)
+    for h in range(3):
+        r = math.exp(slopes[h])
+        for i in range(Sq):
+            q = input_pos + i
+            w = np.array([r ** (q - j) if j <= q else 0.0 for j in range(Sk)])
+            assert np.allclose(O[0, h, i], w / w.sum(), rtol=0, atol=1e-12), (h, i)
+            assert abs(L[0, h, i] - math.log(w.sum())) < 1e-12, (h, i)
+
+
+def pin_flex_document_blocks(orc):
+    """DocumentMask over contiguous documents (ids per position) with the causal
+    mask is block-diagonal: each document's rows equal attention! run on that
+    document alone (its own queries, keys and values, causal, input_pos 0).
+    Also with GQA (4 query heads on 2 KV heads) and a sliding window."""
+    rng = _rng(22)
+    lens = [5, 1, 9, 3, 6]
+    S = sum(lens)
+    doc = np.repeat(np.arange(len(lens)), lens)
+    Q, K, V = rng.standard_normal((2, 4, S, 8)), rng.standard_normal((2, 2, S, 8)), \
+        rng.standard_normal((2, 2, S, 8))
+    for window in (0, 4):
+        O, L = orc.flex_fwd(Q, K, V, 0.35, causal=True, window=window, doc_q=doc, doc_kv=doc)
+        a = 0
+        for n in lens:
+            sl = slice(a, a + n)
+            Od, Ld = orc.attn_fwd(Q[:, :, sl], K[:, :, sl], V[:, :, sl], 0.35, causal=True,
+                                  window=window)
+            assert np.max(np.abs(O[:, :, sl] - Od)) < 1e-12, (window, a, n)
+            assert np.max(np.abs(L[:, :, sl] - Ld)) < 1e-12, (window, a, n)
+            a += n
+
+
 PINS = [
     pin_causal_mask_shape_and_rows,
     pin_sliding_window_rows,
@@ -348,4 +437,8 @@ PINS = [
     pin_row_subset,
     pin_decode_is_last_row_of_prefill,
     pin_decode_closed_forms,
+    pin_flex_golden,
+    pin_flex_softcap_limits,
+    pin_flex_alibi_geometric,
+    pin_flex_document_blocks,
 ]

@@ -40,6 +40,17 @@ MUTANTS = {
                             "out[i * n_kv + j] = (j < offset + i) ? 0.0 : -INFINITY;"),
     "page1_window_wide": ("const int visible = (j <= pos) && (j > pos - window_size);",
                           "const int visible = (j <= pos) && (j >= pos - window_size);"),
+    "flex_softcap_inner": ("sj = softcap * tanh(sj / softcap);", "sj = softcap * tanh(sj);"),
+    "flex_softcap_outer": ("sj = softcap * tanh(sj / softcap);", "sj = tanh(sj / softcap);"),
+    "flex_scale_dropped": ("double sj = scale * dot;", "double sj = dot;"),
+    "flex_alibi_sign": ("(q_pos - (double)j)", "((double)j - q_pos)"),
+    "flex_alibi_kv_head": ("sj += alibi_slopes[hq]", "sj += alibi_slopes[kv_head]"),
+    "flex_doc_ignored": ("if (doc_q[i] != doc_kv[j]) mask[j] = -INFINITY;", "if (0) mask[j] = -INFINITY;"),
+    "flex_doc_kv_by_row": ("if (doc_q[i] != doc_kv[j]) mask[j] = -INFINITY;",
+                           "if (doc_q[i] != doc_kv[i]) mask[j] = -INFINITY;"),
+    "flex_gqa_modulo": ("const long kv_head = hq / group;", "const long kv_head = hq % Hkv;"),
+    "flex_lse_missing_max": ("if (LSE) LSE[row_id] = mx + log(lsum);", "if (LSE) LSE[row_id] = log(lsum);"),
+    "flex_not_normalised": ("const double pj = score[j] / lsum;", "const double pj = score[j];"),
 }
 
 
