@@ -355,6 +355,50 @@ def cpu_baseline(prefill_inputs, dQ, lengths, target_s=12.0, n_seq=2):
     }
 
 
+def time_flex(dev, steps, warmup, peak):
+    """flex_attention! forward rows (soft-cap + document mask, ALiBi): device-resident
+    inputs, CUDA events around each launch; TFLOP/s on the visible pairs."""
+    from gqa_attention_flash_b200 import binding
+    out = {}
+    for key, w in W.FLEX_WORKLOADS.items():
+        Q, K, V, doc, slopes = W.make_flex(w)
+        Qd, Kd, Vd = Q.to(dev), K.to(dev), V.to(dev)
+        O = torch.empty_like(Qd)
+        LSE = torch.empty(Qd.shape[:3], dtype=torch.float32, device=dev)
+        docd = doc.to(dev) if doc is not None else None
+        bm = binding.block_mask_document(w.S, w.S, doc, doc, w.causal).to(dev) \
+            if doc is not None else None
+        sl = slopes.to(dev) if slopes is not None else None
+
+        def run():
+            binding.attn_fwd_flex(O, Qd, Kd, Vd, LSE, w.scale, w.causal, softcap=w.softcap,
+                                  alibi_slopes=sl, doc_q=docd, doc_kv=docd, block_mask=bm)
+        for _ in range(warmup):
+            run()
+        torch.cuda.synchronize()
+        ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+              for _ in range(steps)]
+        for e0, e1 in ev:
+            e0.record()
+            run()
+            e1.record()
+        torch.cuda.synchronize()
+        st = binding.last_device_status()
+        if st != 0:
+            raise RuntimeError(f"flex device status: {binding.status_string(st)}")
+        ms = sum(a.elapsed_time(b) for a, b in ev) / steps
+        flops = w.flops(doc)
+        tf = flops / (ms * 1e-3) / 1e12
+        out[key] = {"workload": w.name, "value": tf, "unit": "TFLOP/s", "ms_per_launch": ms,
+                    "flops_per_launch": flops, "launches": steps,
+                    "roofline": {"bound": "tensor", "achieved": tf, "peak": peak,
+                                 "unit": "TFLOP/s", "frac": tf / peak,
+                                 "kernel": "attn_fwd_kernel<128, flex>"}}
+        del Qd, Kd, Vd, O, LSE
+        torch.cuda.empty_cache()
+    return out
+
+
 def cpu_model():
     try:
         with open("/proc/cpuinfo") as f:
@@ -438,8 +482,11 @@ def main(argv=None):
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
-    ap.add_argument("--only", choices=["prefill", "decode"], default=None,
-                    help="profiling: run one half of the step (no reported number)")
+    ap.add_argument("--no-flex", action="store_true",
+                    help="skip the flex_attention! measurements (reported apart from the step)")
+    ap.add_argument("--only", choices=["prefill", "decode", "flex"], default=None,
+                    help="profiling: run one half of the step, or only the flex_attention! "
+                         "workloads (no reported number)")
     ap.add_argument("--decode-batch", type=int, default=None,
                     help="profiling: smaller decode batch (no reported number)")
     args = ap.parse_args(argv)
@@ -460,6 +507,12 @@ def main(argv=None):
         barrier = lambda: None  # noqa: E731
     dev = torch.device("cuda", local_rank)
     torch.cuda.set_device(dev)
+    if args.only == "flex":
+        peaks, _ = load_peaks()
+        res = time_flex(dev, args.steps, args.warmup, peaks["bf16_tflops"])
+        print(json.dumps({"profiling_run": True,
+                          "flex_ms": {k: v["ms_per_launch"] for k, v in res.items()}}), flush=True)
+        return 0
     step = Step(dev, args.only, args.decode_batch)
     profiling = args.only is not None or args.decode_batch is not None
     sampler = ClockSampler(local_rank)
@@ -525,6 +578,8 @@ def main(argv=None):
         line["e2e"] = e2e
     if world == 1 and not args.no_cpu_baseline:
         line["cpu_baseline"] = cpu_baseline(step.host_prefill, step.dQ_host, step.lengths_host)
+    if not args.no_flex:
+        line["flex"] = time_flex(dev, min(K, 50), args.warmup, peaks["bf16_tflops"])
     print(json.dumps(line), flush=True)
     if world > 1:
         dist.destroy_process_group()

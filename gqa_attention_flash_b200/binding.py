@@ -34,6 +34,14 @@ lib.attn_fwd.restype = _i
 lib.attn_fwd.argtypes = [_p, _p, _p, _p, _p] + [_i] * 6 + [_f, _i, _i, _i, _p, _p]
 lib.attn_fwd_varlen.restype = _i
 lib.attn_fwd_varlen.argtypes = [_p, _p, _p, _p, _p] + [_i] * 6 + [_f, _i, _i, _i, _p, _p, _p]
+lib.attn_fwd_flex.restype = _i
+lib.attn_fwd_flex.argtypes = [_p, _p, _p, _p, _p] + [_i] * 6 + [_f, _i, _i, _i, _p, _p, _f, _p, _p,
+                                                                _p, _p, _p]
+_KEEP = ctypes.CFUNCTYPE(_i, _i, _i, _p)
+lib.attn_block_mask_build.restype = _i
+lib.attn_block_mask_build.argtypes = [_p, _i, _i, _i, _KEEP, _p]
+lib.attn_block_mask_document.restype = _i
+lib.attn_block_mask_document.argtypes = [_p, _i, _i, _i, _i, _i, _p, _p]
 lib.attn_decode.restype = _i
 lib.attn_decode.argtypes = [_p, _p, _p, _p, _p, _i, _p] + [_i] * 5
 lib.attn_decode_noalloc.restype = _i
@@ -88,6 +96,49 @@ def attn_fwd(O, Q, K, V, LSE, scale, causal=False, window=0, input_pos=0, k_leng
     else:
         rc = lib.attn_fwd(*args, _stream(stream))
         _check(rc, "attn_fwd")
+
+
+def attn_fwd_flex(O, Q, K, V, LSE, scale, causal=False, window=0, input_pos=0, k_lengths=None,
+                  q_lengths=None, softcap=0.0, alibi_slopes=None, doc_q=None, doc_kv=None,
+                  block_mask=None, stream=None):
+    """flex_attention! forward: attn_fwd plus SoftCapScore (softcap > 0) or
+    AliBiScore (alibi_slopes, fp32 (Hq,)), DocumentMask (doc_q int32 (Sq,), doc_kv
+    int32 (Sk,)) and a BlockMask (uint8 (ceil(Sq/64), ceil(Sk/64))), all on the
+    device."""
+    B, Hq, Sq, D = Q.shape
+    _, Hkv, Sk, _ = K.shape
+    rc = lib.attn_fwd_flex(_ptr(O), _ptr(Q), _ptr(K), _ptr(V), _ptr(LSE), B, Hq, Hkv, Sq, Sk, D,
+                           float(scale), int(causal), int(window), int(input_pos),
+                           _ptr(k_lengths), _ptr(q_lengths), float(softcap), _ptr(alibi_slopes),
+                           _ptr(doc_q), _ptr(doc_kv), _ptr(block_mask), _stream(stream))
+    _check(rc, "attn_fwd_flex")
+
+
+def block_mask_shape(Sq: int, Sk: int):
+    return ((Sq + 63) // 64, (Sk + 63) // 64)
+
+
+def block_mask_document(Sq, Sk, doc_q, doc_kv, causal=False, window=0, input_pos=0):
+    """Host uint8 BlockMask for DocumentMask (+ causal / window): doc_q, doc_kv are
+    int32 CPU tensors of lengths Sq and Sk.  Returns a CPU uint8 tensor."""
+    out = torch.empty(block_mask_shape(Sq, Sk), dtype=torch.uint8)
+    dq = doc_q.to(torch.int32).contiguous()
+    dk = doc_kv.to(torch.int32).contiguous()
+    assert dq.numel() == Sq and dk.numel() == Sk and not dq.is_cuda and not dk.is_cuda
+    rc = lib.attn_block_mask_document(_ptr(out), int(Sq), int(Sk), int(input_pos), int(causal),
+                                      int(window), _ptr(dq), _ptr(dk))
+    _check(rc, "attn_block_mask_document")
+    return out
+
+
+def block_mask_build(Sq, Sk, keep, input_pos=0):
+    """Host uint8 BlockMask from a Python predicate keep(q, kv) -> bool on absolute
+    query position q and key position kv (the page's build_block_mask)."""
+    out = torch.empty(block_mask_shape(Sq, Sk), dtype=torch.uint8)
+    cb = _KEEP(lambda q, kv, ctx: 1 if keep(q, kv) else 0)
+    rc = lib.attn_block_mask_build(_ptr(out), int(Sq), int(Sk), int(input_pos), cb, None)
+    _check(rc, "attn_block_mask_build")
+    return out
 
 
 def attn_decode(O, Q, K, V, lengths, n_splits=8, stream=None):

@@ -174,6 +174,58 @@ attn_status_t attn_fwd(void *O, const void *Q, const void *K, const void *V, flo
                            input_pos, k_lengths, nullptr, stream);
 }
 
+attn_status_t attn_fwd_flex(void *O, const void *Q, const void *K, const void *V, float *LSE,
+                            int B, int Hq, int Hkv, int Sq, int Sk, int D, float scale,
+                            int causal, int window, int input_pos,
+                            const int32_t *k_lengths, const int32_t *q_lengths,
+                            float softcap, const float *alibi_slopes,
+                            const int32_t *doc_q, const int32_t *doc_kv,
+                            const uint8_t *block_mask, void *stream) {
+    attn_status_t st =
+        validate_fwd(O, Q, K, V, LSE, B, Hq, Hkv, Sq, Sk, D, scale, causal, window, input_pos);
+    if (st != ATTN_OK) return st;
+    if (!(softcap >= 0.f) || !std::isfinite(softcap)) return ATTN_ERR_INVALID;
+    if (softcap > 0.f && alibi_slopes) return ATTN_ERR_INVALID;
+    if ((doc_q == nullptr) != (doc_kv == nullptr)) return ATTN_ERR_INVALID;
+    if ((reinterpret_cast<uintptr_t>(alibi_slopes) | reinterpret_cast<uintptr_t>(doc_q) |
+         reinterpret_cast<uintptr_t>(doc_kv)) & 3u)
+        return ATTN_ERR_INVALID;
+    if ((long long)Sk > (long long)gqa::kFlexMaxKvTiles * 128) return ATTN_ERR_UNSUPPORTED;
+    if ((long long)B * Hq * Sq == 0) return ATTN_OK;
+    FwdArgs a;
+    a.O = O;
+    a.Q = Q;
+    a.K = K;
+    a.V = V;
+    a.LSE = LSE;
+    a.k_lengths = k_lengths;
+    a.q_lengths = q_lengths;
+    a.B = B;
+    a.Hq = Hq;
+    a.Hkv = Hkv;
+    a.Sq = Sq;
+    a.Sk = Sk;
+    a.D = D;
+    a.scale = scale;
+    a.causal = causal;
+    a.window = window;
+    a.input_pos = input_pos;
+    a.flex = 1;
+    a.softcap = softcap;
+    a.alibi_slopes = alibi_slopes;
+    a.doc_q = doc_q;
+    a.doc_kv = doc_kv;
+    a.block_mask = block_mask;
+    if (Sk == 0) {
+        a.K = Q;  // stand-in tensor map; no key is visible
+        a.V = Q;
+        a.doc_kv = nullptr;
+        a.doc_q = nullptr;
+        a.block_mask = nullptr;
+    }
+    return launch_fwd(a, static_cast<cudaStream_t>(stream));
+}
+
 attn_status_t attn_decode(void *O, const void *Q, const void *K, const void *V,
                           const int32_t *lengths, int n_splits, void *stream, int B, int Hq,
                           int Hkv, int S_cap, int D) {

@@ -41,6 +41,7 @@ constexpr int kWarpTma = 8;
 constexpr int kWarpMma = 9;
 constexpr int kThreads = 384;
 constexpr int kLaunchRegs = 168;     // per thread at launch (checked on the host)
+constexpr int kListMax = kFlexMaxKvTiles;  // flex: KV tiles per CTA list
 constexpr uint32_t kProducerRegs = 64;
 constexpr uint32_t kSoftmaxRegs = 216;
 static_assert(128 * kProducerRegs + 256 * kSoftmaxRegs <= kThreads * kLaunchRegs,
@@ -67,6 +68,11 @@ struct FwdCfg {
     static constexpr int N_BARS = 7 + 3 * NS;
     static constexpr int OFF_MISC = OFF_BAR + N_BARS * 8;  // tmem slot, abort flag
     static constexpr int SMEM_BYTES = OFF_MISC + 16 + 1024;  // + alignment slack
+    // flex_attention! only: count + list of the KV tiles the CTA visits
+    // and, per query tile, the entries it uses
+    static constexpr int OFF_LIST = OFF_MISC + 16;
+    static constexpr int OFF_TLIST = OFF_LIST + 4 * (kListMax + 1);  // [2]
+    static constexpr int SMEM_BYTES_FLEX = OFF_TLIST + 2 * 4 * (kListMax + 1) + 1024;
     static constexpr uint32_t TMEM_COLS = 512;
     __host__ __device__ static constexpr uint32_t s_col(int t) { return t * BN; }
     __host__ __device__ static constexpr uint32_t o_col(int t) { return 2 * BN + t * D; }
@@ -82,11 +88,61 @@ struct FwdParams {
     int causal, window, input_pos;
     uint64_t wait_limit_ns;
     int *status;  // device status word
+    // flex_attention! (read only by the flex instantiation)
+    float scale;             // natural-log scale of the scores
+    float softcap;           // > 0: SoftCapScore(cap)
+    float softcap_k;         // 2 log2(e) scale / cap
+    float softcap_c;         // cap log2(e)
+    const float *alibi;      // AliBiScore slopes, one per query head, or null
+    const int32_t *doc_q;    // DocumentMask ids per local query row, or null
+    const int32_t *doc_kv;   // ... per key, or null
+    const uint8_t *bmask;    // BlockMask states of 64x64 blocks (n_qb, n_kb), or null
+    int n_qb, n_kb;
 };
+
+// flex_attention!: 2-bit states of the four 64x64 blocks of the 128x128 tile
+// (query tile qt, KV tile u): 0 = nothing visible, 1 = some pairs visible (apply
+// the document mask), 2 = every pair the block mask covers is visible.  State of
+// block (query half qs, key half ks) sits at bits 2 * (2 qs + ks).  Blocks past
+// the ends of the BlockMask are 0.
+__device__ __forceinline__ uint32_t flex_states(const FwdParams &p, int qt, int u) {
+    uint32_t st = 0;
+#pragma unroll
+    for (int qs = 0; qs < 2; ++qs)
+#pragma unroll
+        for (int ks = 0; ks < 2; ++ks) {
+            const int qb = 2 * qt + qs, kb = 2 * u + ks;
+            uint32_t v = 0;
+            if (qb < p.n_qb && kb < p.n_kb) {
+                if (p.bmask) {
+                    const uint32_t m = p.bmask[(size_t)qb * p.n_kb + kb];
+                    v = m == 0 ? 0u : (m == 2 ? 2u : 1u);
+                } else {
+                    v = p.doc_q ? 1u : 2u;
+                }
+            }
+            st |= v << (2 * (2 * qs + ks));
+        }
+    return st;
+}
+
+// SoftCapScore in log2 units for a raw dot product d (s = scale d):
+//   cap tanh(s / cap) log2e,  tanh|y| = 1 - 2 / (e^{2|y|} + 1),
+// with k = 2 log2e scale / cap (so e^{2|y|} = 2^{k |d|}) and c = cap log2e.
+__device__ __forceinline__ float softcap_score(float d, float k, float c) {
+    const float e = fast_exp2(fabsf(d) * k);
+    float r;
+    asm("rcp.approx.ftz.f32 %0, %1;" : "=f"(r) : "f"(e + 1.f));
+    return copysignf(fmaf(-2.f * c, r, c), d);
+}
 
 __device__ __forceinline__ float neg_inf() { return __int_as_float(0xff800000); }
 
-template <int D>
+// kMode: score mod of flex_attention!: 0 = none, 2 = SoftCapScore, 3 = AliBiScore.
+// kList: the CTA visits the KV tiles of a per-CTA list built from the BlockMask
+// and applies the block states / DocumentMask per element; without it, the KV
+// tiles of the analytic ranges in order (attention! is <D, 0, false>).
+template <int D, int kMode, bool kList>
 __global__ void __launch_bounds__(kThreads, 1)
     attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                     const __grid_constant__ CUtensorMap tmV, const FwdParams p) {
@@ -156,6 +212,13 @@ __global__ void __launch_bounds__(kThreads, 1)
 #define TILE_LO(t) ((t) ? lo1 : lo0)
 #define TILE_HI(t) ((t) ? hi1 : hi0)
 #define USES(t, u) ((u) >= TILE_LO(t) && (u) < TILE_HI(t))
+    // flex: [0] = number of KV tiles the CTA visits, then one entry per tile:
+    // bits 0-15 the KV tile index, bits 16-23 / 24-31 the block states of query
+    // tile 0 / 1 (0 when that query tile skips the KV tile).
+    uint32_t *kv_list = reinterpret_cast<uint32_t *>(smem + C::OFF_LIST);
+    // per query tile t: [0] = count, then entries g | u << 10 | states << 20 |
+    // (query tile 0 uses it) << 28, in visiting order
+    uint32_t *tile_list = reinterpret_cast<uint32_t *>(smem + C::OFF_TLIST);
 
     // ---- set-up ----
     if (threadIdx.x == 0) {
@@ -173,6 +236,65 @@ __global__ void __launch_bounds__(kThreads, 1)
         *abort_flag = 0;
         fence_mbar_init();
     }
+    // AliBiScore with a negative slope: the bias grows towards the query, so the
+    // KV tiles are visited nearest first; the running max is then found at once
+    // and the lazy rescale of O stays rare.  (The softmax does not depend on the
+    // visiting order.)
+    bool rev = false;
+    if constexpr (kMode == 3) rev = p.alibi[hq] < 0.f;
+    if constexpr (kList) {
+        // The KV tiles this CTA visits: inside a query tile's analytic range and
+        // holding a visible block (BlockMask of flex_attention!), in order.
+        if (warp == kWarpTma) {
+            int count = 0;
+            for (int base = u_lo; n_u > 0 && base < u_hi; base += 32) {
+                const int u = base + lane;
+                uint32_t e = 0;
+                if (u < u_hi) {
+                    const uint32_t s0 = USES(0, u) ? flex_states(p, pair * kTiles, u) : 0u;
+                    const uint32_t s1 = USES(1, u) ? flex_states(p, pair * kTiles + 1, u) : 0u;
+                    if (s0 | s1) e = static_cast<uint32_t>(u) | (s0 << 16) | (s1 << 24);
+                }
+                const uint32_t vote = __ballot_sync(0xffffffffu, e != 0);
+                if (e != 0) kv_list[1 + count + __popc(vote & ((1u << lane) - 1u))] = e;
+                count += __popc(vote);
+            }
+            if constexpr (kMode == 3) {
+                if (rev) {
+                    __syncwarp();
+                    for (int j = lane; j < count / 2; j += 32) {
+                        const uint32_t x = kv_list[1 + j];
+                        kv_list[1 + j] = kv_list[count - j];
+                        kv_list[count - j] = x;
+                    }
+                    __syncwarp();
+                }
+            }
+            __syncwarp();
+#pragma unroll
+            for (int t = 0; t < kTiles; ++t) {
+                uint32_t *tl = tile_list + t * (kListMax + 1);
+                int n_t_list = 0;
+                for (int base = 0; base < count; base += 32) {
+                    const int g = base + lane;
+                    uint32_t x = 0;
+                    bool use = false;
+                    if (g < count) {
+                        const uint32_t e = kv_list[1 + g];
+                        const uint32_t st = (e >> (16 + 8 * t)) & 0xFFu;
+                        use = st != 0;
+                        x = static_cast<uint32_t>(g) | ((e & 0x3FFu) << 10) | (st << 20) |
+                            ((((e >> 16) & 0xFFu) != 0 ? 1u : 0u) << 28);
+                    }
+                    const uint32_t vote = __ballot_sync(0xffffffffu, use);
+                    if (use) tl[1 + n_t_list + __popc(vote & ((1u << lane) - 1u))] = x;
+                    n_t_list += __popc(vote);
+                }
+                if (lane == 0) tl[0] = static_cast<uint32_t>(n_t_list);
+            }
+            if (lane == 0) kv_list[0] = static_cast<uint32_t>(count);
+        }
+    }
     if (warp == kWarpMma) {
         tmem_alloc(smem_u32(tmem_slot), C::TMEM_COLS);
         tmem_relinquish();
@@ -186,7 +308,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       regs_dec<kProducerRegs>();
       if (warp == kWarpTma) {
         // ===================== TMA producer =====================
-        if (lane == 0 && n_u > 0) {
+        const int n_load = kList ? static_cast<int>(kv_list[0]) : n_u;
+        if (lane == 0 && n_load > 0) {
             prefetch_tensormap(&tmQ);
             prefetch_tensormap(&tmK);
             prefetch_tensormap(&tmV);
@@ -199,13 +322,15 @@ __global__ void __launch_bounds__(kThreads, 1)
                     tma_load_3d(sbase + C::OFF_Q + t * C::Q_BYTES + c * C::BOX, &tmQ, bar(C::BAR_Q),
                                 c * 64, (pair * kTiles + t) * BM, b * p.Hq + hq);
             }
-            for (int g = 0; g < n_u; ++g) {
+            for (int g = 0; g < n_load; ++g) {
                 const int st = g % C::NS;
                 const int use = g / C::NS;
                 if (use > 0 &&
                     !mbar_wait(bar(C::BAR_EMPTY + st), (use - 1) & 1, abort_flag, p.wait_limit_ns, p.status))
                     break;
-                const int kv_row = (u_lo + g) * BN;
+                const int kv_row =
+                    (kList ? static_cast<int>(kv_list[1 + g] & 0xFFFFu)
+                           : (rev ? u_hi - 1 - g : u_lo + g)) * BN;
                 mbar_arrive_expect_tx(bar(C::BAR_KFULL + st), C::KV_BYTES);
                 for (int c = 0; c < C::NBOX; ++c)
                     tma_load_3d(sbase + C::OFF_K + st * C::KV_BYTES + c * C::BOX, &tmK,
@@ -218,11 +343,13 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
       } else if (warp == kWarpMma) {
         // ===================== MMA issuer =====================
-        if (lane == 0 && n_u > 0) {
+        const int n_load = kList ? static_cast<int>(kv_list[0]) : n_u;
+        if (lane == 0 && n_load > 0) {
             constexpr uint32_t idS = idesc_bf16_f32(BM, BN, 0, 0);
             constexpr uint32_t idO = idesc_bf16_f32(BM, D, 0, 1);
-            auto issue_s = [&](int t, int u) -> bool {
-                const int g = u - u_lo;
+            // g: index of the KV tile in the CTA's load order; i: the query tile's
+            // own iteration index.
+            auto issue_s = [&](int t, int g) -> bool {
                 const int st = g % C::NS;
                 if (!mbar_wait(bar(C::BAR_KFULL + st), (g / C::NS) & 1, abort_flag,
                                p.wait_limit_ns, p.status))
@@ -239,10 +366,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                 mma_commit(bar(C::BAR_SFULL + t));
                 return true;
             };
-            auto issue_pv = [&](int t, int u) -> bool {
-                const int g = u - u_lo;
+            auto issue_pv = [&](int t, int g, int i) -> bool {
                 const int st = g % C::NS;
-                const int i = u - TILE_LO(t);  // this tile's iteration index
                 if (!mbar_wait(bar(C::BAR_PFULL + t), i & 1, abort_flag, p.wait_limit_ns, p.status))
                     return false;
                 if (!mbar_wait(bar(C::BAR_VFULL + st), (g / C::NS) & 1, abort_flag,
@@ -259,16 +384,43 @@ __global__ void __launch_bounds__(kThreads, 1)
                 return true;
             };
             bool ok = mbar_wait(bar(C::BAR_Q), 0, abort_flag, p.wait_limit_ns, p.status);
+            if constexpr (!kList) {
+                const int u_first = rev ? u_hi - 1 : u_lo;
 #pragma unroll
-            for (int t = 0; t < kTiles; ++t)
-                if (ok && USES(t, u_lo)) ok = issue_s(t, u_lo);
-            for (int u = u_lo; ok && u < u_hi; ++u) {
+                for (int t = 0; t < kTiles; ++t)
+                    if (ok && USES(t, u_first)) ok = issue_s(t, 0);
+                for (int g = 0; ok && g < n_u; ++g) {
+                    const int u = rev ? u_hi - 1 - g : u_lo + g;
+                    const int un = rev ? u - 1 : u + 1;
 #pragma unroll
-                for (int t = 0; t < kTiles; ++t) {
-                    if (ok && USES(t, u)) ok = issue_pv(t, u);
-                    if (ok && u + 1 < u_hi && USES(t, u + 1)) ok = issue_s(t, u + 1);
+                    for (int t = 0; t < kTiles; ++t) {
+                        if (ok && USES(t, u))
+                            ok = issue_pv(t, g, rev ? TILE_HI(t) - 1 - u : u - TILE_LO(t));
+                        if (ok && g + 1 < n_u && USES(t, un)) ok = issue_s(t, g + 1);
+                    }
+                    if (ok) mma_commit(bar(C::BAR_EMPTY + g % C::NS));
                 }
-                if (ok) mma_commit(bar(C::BAR_EMPTY + (u - u_lo) % C::NS));
+            } else {
+                // Same order over the listed KV tiles: P_t V_g, then S_t for the next
+                // listed tile when tile t uses it; a tile that resumes after a gap
+                // issues its S when its next listed tile comes up.
+                int it0 = 0, it1 = 0;
+                bool sq0 = false, sq1 = false;  // S of tile t already issued for this g
+                for (int g = 0; ok && g < n_load; ++g) {
+                    const uint32_t e = kv_list[1 + g];
+                    const uint32_t en = g + 1 < n_load ? kv_list[2 + g] : 0u;
+#pragma unroll
+                    for (int t = 0; t < kTiles; ++t) {
+                        if (!ok || ((e >> (16 + 8 * t)) & 0xFFu) == 0) continue;
+                        if (!(t ? sq1 : sq0)) ok = issue_s(t, g);
+                        if (ok) ok = issue_pv(t, g, t ? it1 : it0);
+                        if (t) ++it1; else ++it0;
+                        const bool next = ok && ((en >> (16 + 8 * t)) & 0xFFu) != 0;
+                        if (next) ok = issue_s(t, g + 1);
+                        if (t) sq1 = next; else sq0 = next;
+                    }
+                    if (ok) mma_commit(bar(C::BAR_EMPTY + g % C::NS));
+                }
             }
         }
       }
@@ -287,16 +439,47 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int my_lo = TILE_LO(t);
         const int my_hi = TILE_HI(t);
         const int my_qlast = t ? ql1 : ql0;
-        const int n_t = my_hi > my_lo ? my_hi - my_lo : 0;
         const uint32_t bar_s = bar(C::BAR_SFULL + t), bar_p = bar(C::BAR_PFULL + t),
                        bar_o = bar(C::BAR_ODONE + t);
         float m_used = neg_inf();  // max subtracted so far (log2 units)
         float l = 0.f;
         bool ok = true;
+        // flex: score scale folded into the scores before the max, so the
+        // exponent below uses a unit factor
+        const float sl2 = kMode >= 2 ? 1.f : p.scale_log2;
+        int doc_row = -1;
+        if constexpr (kList) {
+            if (p.doc_q && row < p.Sq) doc_row = p.doc_q[row];
+        }
+        // AliBiScore in log2 units: s * scale * log2e + slope * log2e * (pos - kv0 - c)
+        float al_a = 0.f, al_b = 0.f;
+        if constexpr (kMode == 3) {
+            al_b = p.alibi[hq] * 1.4426950408889634f;
+            al_a = p.scale_log2;
+        }
 
-        for (int i = 0; i < n_t; ++i) {
-            const int u = my_lo + i;
-            const int g = u - u_lo;
+        // KV tiles of this query tile: its analytic range, or (flex) the listed
+        // tiles whose block states for this query tile are not all 0.
+        const uint32_t *my_list = tile_list + t * (kListMax + 1);
+        const int n_iter = kList ? static_cast<int>(my_list[0]) : (my_hi > my_lo ? my_hi - my_lo : 0);
+        int n_done = 0;  // KV tiles this query tile has processed
+        for (int it = 0; it < n_iter; ++it) {
+            int u, g, i;  // KV tile, its load index, this query tile's iteration
+            uint32_t my_st = 0;
+            bool tile0_uses;  // query tile 0 also visits this KV tile
+            if constexpr (kList) {
+                const uint32_t e = my_list[1 + it];
+                g = static_cast<int>(e & 0x3FFu);
+                u = static_cast<int>((e >> 10) & 0x3FFu);
+                my_st = (e >> 20) & 0xFFu;
+                tile0_uses = (e >> 28) != 0;
+                i = it;
+            } else {
+                u = rev ? my_hi - 1 - it : my_lo + it;
+                g = rev ? u_hi - 1 - u : u - u_lo;
+                i = it;
+                tile0_uses = USES(0, u);
+            }
             const int kv0 = u * BN;
             if (!warp_wait(bar_s, i & 1, abort_flag, p.wait_limit_ns, p.status)) {
                 ok = false;
@@ -310,19 +493,73 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
             for (int c = 0; c < 4; ++c) reg_fence32(sr[c]);
             float *s = reinterpret_cast<float *>(&sr[0][0]);
+            // flex_attention! score mods on s = scale <q, k>, then log2 units
+            if constexpr (kMode == 2) {
+                // 16 columns at a time: the fence after each group also redefines the
+                // next group's inputs, so at most 16 elements' temporaries are live
+                uint32_t *flat = &sr[0][0];
+#pragma unroll
+                for (int gp = 0; gp < BN / 16; ++gp) {
+#pragma unroll
+                    for (int c = 16 * gp; c < 16 * gp + 16; ++c)
+                        s[c] = softcap_score(s[c], p.softcap_k, p.softcap_c);
+                    const int f0 = gp < BN / 16 - 1 ? 16 * gp : BN - 32;
+                    reg_fence32(*reinterpret_cast<uint32_t(*)[32]>(flat + f0));
+                }
+            } else if constexpr (kMode == 3) {
+                const float t0 = al_b * static_cast<float>(pos - kv0);  // bias of key kv0
+#pragma unroll
+                for (int c = 0; c < BN; ++c)
+                    s[c] = fmaf(s[c], al_a, fmaf(-al_b, static_cast<float>(c), t0));
+            }
             // step a5: per-element mask on boundary tiles only
             const bool edge = (kv0 + BN > k_end) ||
                               (p.causal && (long long)kv0 + BN - 1 > (long long)p.input_pos + q0) ||
                               (p.window > 0 &&
-                               (long long)kv0 <= (long long)p.input_pos + my_qlast - p.window);
+                               (long long)kv0 <= (long long)p.input_pos + my_qlast - p.window) ||
+                              (kList && my_st != 0xAAu);
             if (edge) {
                 long long hi = k_end;
                 if (p.causal) hi = min(hi, pos + 1);
                 const long long lo = p.window > 0 ? pos - p.window + 1 : 0;
                 const int c_hi = static_cast<int>(max(-1ll, min((long long)BN, hi - kv0)));
                 const int c_lo = static_cast<int>(max(-1ll, min((long long)BN, lo - kv0)));
+                if constexpr (kList) {
+                    // One visibility bit per key, 32 keys per word: the analytic range,
+                    // the block state of this row's 64-row half for the key's half
+                    // (0: none, 2: all), and for state 1 the document ids.  The ids
+                    // of the tile's keys are read once per warp (one per lane) and
+                    // passed around with shuffles; this keeps the unrolled per-key
+                    // code as small as the plain path's.
+                    const uint32_t qs = static_cast<uint32_t>(r >> 6);
+                    uint32_t vm[4];
 #pragma unroll
-                for (int c = 0; c < BN; ++c) s[c] = (c >= c_lo && c < c_hi) ? s[c] : neg_inf();
+                    for (int j = 0; j < 4; ++j) {
+                        const int lo_j = min(max(c_lo - 32 * j, 0), 32);
+                        const int hi_j = min(max(c_hi - 32 * j, 0), 32);
+                        const uint32_t below_hi = hi_j >= 32 ? 0xffffffffu : ((1u << hi_j) - 1u);
+                        const uint32_t below_lo = lo_j >= 32 ? 0xffffffffu : ((1u << lo_j) - 1u);
+                        uint32_t m = below_hi & ~below_lo;
+                        const uint32_t st = (my_st >> (4 * qs + 2 * (j >> 1))) & 3u;
+                        if (st == 0) m = 0;
+                        if (st == 1 && p.doc_kv) {  // uniform: st depends on the warp only
+                            const int kc = kv0 + 32 * j + lane;
+                            const int dv = kc < p.Sk ? p.doc_kv[kc] : 0;
+                            uint32_t same = 0;
+#pragma unroll 1
+                            for (int c = 0; c < 32; ++c)
+                                same |= (__shfl_sync(0xffffffffu, dv, c) == doc_row ? 1u : 0u) << c;
+                            m &= same;
+                        }
+                        vm[j] = m;
+                    }
+#pragma unroll
+                    for (int c = 0; c < BN; ++c)
+                        s[c] = ((vm[c >> 5] >> (c & 31)) & 1u) ? s[c] : neg_inf();
+                } else {
+#pragma unroll
+                    for (int c = 0; c < BN; ++c) s[c] = (c >= c_lo && c < c_hi) ? s[c] : neg_inf();
+                }
             }
             // step a6: online softmax in the exp2 domain with lazy rescaling
             float mx0 = s[0], mx1 = s[1];
@@ -331,7 +568,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 mx0 = fmaxf(mx0, s[c]);
                 mx1 = fmaxf(mx1, s[c + 1]);
             }
-            const float m_new = fmaxf(mx0, mx1) * p.scale_log2;
+            const float m_new = fmaxf(mx0, mx1) * sl2;
             float alpha = 1.f;
             bool resc = false;
             if (m_new > m_used + 8.f) {
@@ -346,8 +583,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                 uint32_t pk[16];
 #pragma unroll
                 for (int k = 0; k < 16; ++k) {
-                    const float p0 = fast_exp2(fmaf(s[c * 32 + 2 * k], p.scale_log2, neg_m));
-                    const float p1 = fast_exp2(fmaf(s[c * 32 + 2 * k + 1], p.scale_log2, neg_m));
+                    const float p0 = fast_exp2(fmaf(s[c * 32 + 2 * k], sl2, neg_m));
+                    const float p1 = fast_exp2(fmaf(s[c * 32 + 2 * k + 1], sl2, neg_m));
                     sum0 += p0;
                     sum1 += p1;
                     pk[k] = pack_bf16x2(p0, p1);
@@ -373,7 +610,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             // Key rows at or past k_end inside this tile may hold anything; their
             // weights are exactly 0, but 0 * NaN is NaN, so zero those V rows (done
             // by the first query tile that uses this KV tile).
-            if (k_end < p.Sk && k_end > kv0 && k_end < kv0 + BN && (t == 0 || !USES(0, u))) {
+            if (k_end < p.Sk && k_end > kv0 && k_end < kv0 + BN && (t == 0 || !tile0_uses)) {
                 const int st = g % C::NS;
                 if (!warp_wait(bar(C::BAR_VFULL + st), (g / C::NS) & 1, abort_flag,
                                p.wait_limit_ns, p.status)) {
@@ -396,13 +633,14 @@ __global__ void __launch_bounds__(kThreads, 1)
             tc_fence_before();
             mbar_arrive(bar_p);
             if (!ok) break;
+            n_done = i + 1;
         }
 
         // step a8: epilogue
         const bool row_in = row < p.Sq;
-        bool have = ok && n_t > 0;
+        bool have = ok && n_done > 0;
         if (have &&
-            !warp_wait(bar_o, (n_t - 1) & 1, abort_flag, p.wait_limit_ns, p.status))
+            !warp_wait(bar_o, (n_done - 1) & 1, abort_flag, p.wait_limit_ns, p.status))
             have = false;
         const bool out_valid = have && row < q_end && l > 0.f;
         const float inv_l = out_valid ? 1.f / l : 0.f;
@@ -453,9 +691,10 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
 }
 
-template <int D>
+template <int D, int kMode, bool kList>
 attn_status_t launch_fwd_d(const FwdArgs &a, cudaStream_t stream) {
     using C = FwdCfg<D>;
+    constexpr int kSmem = kList ? C::SMEM_BYTES_FLEX : C::SMEM_BYTES;
     CUtensorMap tq, tk, tv;
     attn_status_t st;
     if ((st = make_tmap_bf16_3d(&tq, a.Q, D, a.Sq, (uint64_t)a.B * a.Hq, BM)) != ATTN_OK) return st;
@@ -466,11 +705,11 @@ attn_status_t launch_fwd_d(const FwdArgs &a, cudaStream_t stream) {
         // The register hand-over inside the kernel assumes exactly kLaunchRegs
         // registers per thread at launch; refuse to launch a build where it differs.
         cudaFuncAttributes fa;
-        if (cudaFuncGetAttributes(&fa, attn_fwd_kernel<D>) != cudaSuccess ||
+        if (cudaFuncGetAttributes(&fa, attn_fwd_kernel<D, kMode, kList>) != cudaSuccess ||
             fa.numRegs != kLaunchRegs)
             return ATTN_ERR_CUDA;
-        if (cudaFuncSetAttribute(attn_fwd_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 C::SMEM_BYTES) != cudaSuccess)
+        if (cudaFuncSetAttribute(attn_fwd_kernel<D, kMode, kList>,
+                                 cudaFuncAttributeMaxDynamicSharedMemorySize, kSmem) != cudaSuccess)
             return ATTN_ERR_CUDA;
         configured = true;
     }
@@ -492,20 +731,44 @@ attn_status_t launch_fwd_d(const FwdArgs &a, cudaStream_t stream) {
     p.input_pos = a.input_pos;
     p.wait_limit_ns = kWaitLimitNs;
     p.status = device_status_word();
+    p.scale = a.scale;
+    p.softcap = a.softcap;
+    p.softcap_k = a.softcap > 0.f ? 2.8853900817779268f * a.scale / a.softcap : 0.f;
+    p.softcap_c = a.softcap * 1.4426950408889634f;
+    p.alibi = a.alibi_slopes;
+    p.doc_q = a.doc_q;
+    p.doc_kv = a.doc_kv;
+    p.bmask = a.block_mask;
+    p.n_qb = (a.Sq + 63) / 64;
+    p.n_kb = (a.Sk + 63) / 64;
     if (!p.status) return ATTN_ERR_CUDA;
     const long long grid = (long long)p.n_pairs * a.Hq * a.B;
     if (grid == 0) return ATTN_OK;
     if (grid > 0x7fffffffll) return ATTN_ERR_INVALID;
-    attn_fwd_kernel<D><<<static_cast<unsigned>(grid), kThreads, C::SMEM_BYTES, stream>>>(tq, tk, tv,
-                                                                                          p);
+    attn_fwd_kernel<D, kMode, kList>
+        <<<static_cast<unsigned>(grid), kThreads, kSmem, stream>>>(tq, tk, tv, p);
     return cudaGetLastError() == cudaSuccess ? ATTN_OK : ATTN_ERR_CUDA;
 }
 
 }  // namespace
 
 attn_status_t launch_fwd(const FwdArgs &a, cudaStream_t stream) {
-    if (a.D == 128) return launch_fwd_d<128>(a, stream);
-    if (a.D == 64) return launch_fwd_d<64>(a, stream);
+    const int mode = !a.flex ? 0 : (a.softcap > 0.f ? 2 : (a.alibi_slopes ? 3 : 0));
+    const bool list = a.flex && (a.block_mask || a.doc_q);
+#define GQA_LAUNCH(DD)                                                            \
+    do {                                                                          \
+        if (list) {                                                               \
+            if (mode == 0) return launch_fwd_d<DD, 0, true>(a, stream);           \
+            if (mode == 2) return launch_fwd_d<DD, 2, true>(a, stream);           \
+            return launch_fwd_d<DD, 3, true>(a, stream);                          \
+        }                                                                         \
+        if (mode == 0) return launch_fwd_d<DD, 0, false>(a, stream);              \
+        if (mode == 2) return launch_fwd_d<DD, 2, false>(a, stream);              \
+        return launch_fwd_d<DD, 3, false>(a, stream);                             \
+    } while (0)
+    if (a.D == 128) GQA_LAUNCH(128);
+    if (a.D == 64) GQA_LAUNCH(64);
+#undef GQA_LAUNCH
     return ATTN_ERR_UNSUPPORTED;
 }
 

@@ -22,7 +22,17 @@ struct FwdArgs {
     int B, Hq, Hkv, Sq, Sk, D;
     float scale;
     int causal, window, input_pos;
+    // flex_attention! extras; flex = 0 selects the plain kernel
+    int flex = 0;
+    float softcap = 0.f;
+    const float *alibi_slopes = nullptr;
+    const int32_t *doc_q = nullptr, *doc_kv = nullptr;
+    const uint8_t *block_mask = nullptr;
 };
+
+// Longest KV sequence the flex kernel takes, in 128-key tiles (its per-CTA list
+// of visited tiles lives in shared memory).
+constexpr int kFlexMaxKvTiles = 1024;
 
 struct DecodeArgs {
     void *O;

@@ -88,6 +88,52 @@ DECODE = DecodeWorkload("split-KV decode B64 Hq32 Hkv8 D128 cap32768 n_splits8",
 PREFILL_WORKLOADS = {"tiny": TINY, "llm": LLM, "window": WINDOW, "image": IMAGE}
 
 
+@dataclass(frozen=True)
+class FlexWorkload:
+    """flex_attention! forward workload: a prefill shape plus one score mod and,
+    optionally, packed documents (DocumentMask with a BlockMask)."""
+    name: str
+    B: int
+    Hq: int
+    Hkv: int
+    S: int
+    D: int
+    causal: bool
+    softcap: float = 0.0
+    alibi: bool = False
+    doc_len: tuple | None = None          # (min, max) document length, packed to S
+    seed: int = 0
+
+    @property
+    def scale(self) -> float:
+        return 1.0 / math.sqrt(self.D)
+
+    def flops(self, doc=None) -> int:
+        """4 * D * visible (query, key) pairs, summed over heads and batch."""
+        if doc is None:
+            pairs = self.S * (self.S + 1) // 2 if self.causal else self.S * self.S
+        else:
+            n = torch.bincount(doc.to(torch.int64)).to(torch.int64)
+            pairs = int((n * (n + 1) // 2).sum()) if self.causal else int((n * n).sum())
+        return 4 * self.D * self.Hq * self.B * pairs
+
+
+FLEX_DOC = FlexWorkload("document-masked causal prefill, soft-cap 50: B1 Hq32 Hkv8 S16384 D128, "
+                        "documents 256..4096", 1, 32, 8, 16384, 128, True, softcap=50.0,
+                        doc_len=(256, 4096), seed=5)
+FLEX_ALIBI = FlexWorkload("ALiBi causal prefill B4 Hq32 Hkv8 S4096 D128", 4, 32, 8, 4096, 128,
+                          True, alibi=True, seed=6)
+FLEX_WORKLOADS = {"doc_softcap": FLEX_DOC, "alibi": FLEX_ALIBI}
+
+
+def make_flex(w: FlexWorkload):
+    """CPU inputs of a flex workload: (Q, K, V, doc ids or None, ALiBi slopes or None)."""
+    Q, K, V = random_prefill(w.seed, w.B, w.Hq, w.Hkv, w.S, w.S, w.D)
+    doc = document_ids(w.S, w.seed, *w.doc_len) if w.doc_len else None
+    slopes = alibi_slopes(w.Hq, w.seed) if w.alibi else None
+    return Q, K, V, doc, slopes
+
+
 def visible_pairs(w: PrefillWorkload, k_lengths=None, q_lengths=None) -> int:
     """Number of (query row, key) pairs one query head sees, summed over batch.
 
@@ -149,6 +195,31 @@ def random_prefill(seed, B, Hq, Hkv, Sq, Sk, D):
     K = torch.randn(B, Hkv, Sk, D, generator=g).to(torch.bfloat16)
     V = torch.randn(B, Hkv, Sk, D, generator=g).to(torch.bfloat16)
     return Q, K, V
+
+
+def document_ids(total: int, seed: int, min_len: int = 1, max_len: int = 512, align: int = 1):
+    """int32 (total,) document ids of packed documents: consecutive runs with
+    lengths drawn uniformly from [min_len, max_len] (multiples of ``align``),
+    the last one cut at ``total`` (the DocumentMask workloads)."""
+    g = torch.Generator(device="cpu").manual_seed(seed)
+    ids = torch.empty(total, dtype=torch.int32)
+    pos, d = 0, 0
+    lo, hi = max(1, min_len // align), max(1, max_len // align)
+    while pos < total:
+        n = int(torch.randint(lo, hi + 1, (1,), generator=g)) * align
+        ids[pos:pos + n] = d
+        pos += n
+        d += 1
+    return ids
+
+
+def alibi_slopes(Hq: int, seed: int):
+    """fp32 (Hq,) ALiBi slopes: the geometric family -2^(-8 (h+1) / Hq) of the
+    ALiBi paper with a random sign flip per head, so both signs are exercised."""
+    g = torch.Generator(device="cpu").manual_seed(seed)
+    mag = torch.tensor([2.0 ** (-8.0 * (h + 1) / Hq) for h in range(Hq)], dtype=torch.float32)
+    sign = torch.where(torch.rand(Hq, generator=g) < 0.5, -1.0, 1.0)
+    return (mag * sign).to(torch.float32)
 
 
 def decode_query_and_lengths(w: DecodeWorkload):

@@ -97,6 +97,63 @@ attn_status_t attn_fwd_varlen(void *O, const void *Q, const void *K, const void 
                               void *stream);
 
 /*
+ * attn_fwd_flex -- flex_attention! forward with one score mod and a document
+ * mask (Tylo.jl "Primitives" page, entries `flex_attention!`,
+ * `SoftCapScore`, `AliBiScore`, `DocumentMask`, `BlockMask`).
+ *
+ * Same tensors, masks and lengths as attn_fwd_varlen; on top of them, with
+ * s = scale * <q_i, k_j> the scaled score of query row i and key j:
+ *   softcap       > 0: s -> softcap * tanh(s / softcap)        (SoftCapScore)
+ *   alibi_slopes  float32 (Hq,) device array or NULL:
+ *                 s -> s + alibi_slopes[h] * ((input_pos + i) - j)  (AliBiScore)
+ *                 At most one of softcap > 0 and alibi_slopes is given.
+ *   doc_q, doc_kv int32 device arrays, (Sq,) ids of the query rows and (Sk,)
+ *                 ids of the keys, both NULL or both given: the pair attends
+ *                 only if the ids match (DocumentMask; shared by every batch
+ *                 entry and head).
+ *   block_mask    uint8 device array (ceil(Sq/64), ceil(Sk/64)) or NULL, one
+ *                 state per 64x64 block of (query row, key): 0 = no pair of
+ *                 the block attends (skipped), 2 = every pair attends (document
+ *                 ids not checked), anything else = check each pair.  Build it
+ *                 with attn_block_mask_document or attn_block_mask_build (the
+ *                 page's build_block_mask); it must agree with the other masks.
+ * Limits: Sk <= 131072.  Errors as attn_fwd, plus ATTN_ERR_INVALID for a
+ * negative or non-finite softcap, softcap together with ALiBi, or only one of
+ * doc_q / doc_kv, and ATTN_ERR_UNSUPPORTED for a longer Sk.
+ */
+attn_status_t attn_fwd_flex(void *O, const void *Q, const void *K, const void *V, float *LSE,
+                            int B, int Hq, int Hkv, int Sq, int Sk, int D, float scale,
+                            int causal, int window, int input_pos,
+                            const int32_t *k_lengths, const int32_t *q_lengths,
+                            float softcap, const float *alibi_slopes,
+                            const int32_t *doc_q, const int32_t *doc_kv,
+                            const uint8_t *block_mask, void *stream);
+
+/*
+ * attn_block_mask_build -- the page's build_block_mask (Tylo.jl "Primitives"
+ * page, entry `build_block_mask`, TILE_M = TILE_N = 64) on the host.
+ *
+ *   out   [out] host uint8 (ceil(Sq/64), ceil(Sk/64)), caller-owned.  Block
+ *         (qb, kb) gets 0 if keep is false for every (query row, key) pair of
+ *         the block, 2 if it is true for every pair, 1 otherwise (pairs past
+ *         Sq or Sk are not part of a block).
+ *   keep  predicate on (q, kv): q = input_pos + i is the absolute position of
+ *         query row i, kv the key position; nonzero = attend.
+ * Returns ATTN_ERR_NULL / ATTN_ERR_INVALID on bad arguments.
+ */
+attn_status_t attn_block_mask_build(uint8_t *out, int Sq, int Sk, int input_pos,
+                                    int (*keep)(int q, int kv, void *ctx), void *ctx);
+
+/*
+ * attn_block_mask_document -- attn_block_mask_build for the predicate
+ * "doc_q[i] == doc_kv[kv], and the causal / window rule of attn_fwd holds"
+ * (DocumentMask combined with CausalMask / the sliding window), with host
+ * arrays doc_q (Sq,) and doc_kv (Sk,).
+ */
+attn_status_t attn_block_mask_document(uint8_t *out, int Sq, int Sk, int input_pos, int causal,
+                                       int window, const int32_t *doc_q, const int32_t *doc_kv);
+
+/*
  * attn_decode -- split-KV (Flash-Decoding) attention of one new query token per
  * head and sequence against a KV cache.
  *

@@ -5,6 +5,7 @@ import ctypes
 import os
 import re
 
+import numpy as np
 import pytest
 
 ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
@@ -95,3 +96,70 @@ def test_decode_host_validation(binding):
 def test_bounded_wait_argument_range(binding):
     assert binding.lib.attn_check_bounded_wait(0, None) == 2
     assert binding.lib.attn_check_bounded_wait(3_000_000, None) == 2
+
+
+def flex(binding, **kw):
+    a = dict(O=P, Q=P, K=P, V=P, LSE=None, B=1, Hq=2, Hkv=1, Sq=4, Sk=4, D=128, scale=0.1,
+             causal=1, window=0, input_pos=0, k_lengths=None, q_lengths=None, softcap=0.0,
+             alibi=None, doc_q=None, doc_kv=None, block_mask=None)
+    a.update(kw)
+    return binding.lib.attn_fwd_flex(a["O"], a["Q"], a["K"], a["V"], a["LSE"], a["B"], a["Hq"],
+                                     a["Hkv"], a["Sq"], a["Sk"], a["D"], a["scale"], a["causal"],
+                                     a["window"], a["input_pos"], a["k_lengths"], a["q_lengths"],
+                                     a["softcap"], a["alibi"], a["doc_q"], a["doc_kv"],
+                                     a["block_mask"], None)
+
+
+def test_flex_host_validation(binding):
+    assert flex(binding, Hq=3, Hkv=2) == 2
+    assert flex(binding, D=96) == 3
+    assert flex(binding, softcap=-1.0) == 2
+    assert flex(binding, softcap=float("inf")) == 2
+    assert flex(binding, softcap=float("nan")) == 2
+    assert flex(binding, softcap=5.0, alibi=P) == 2      # one score mod per call
+    assert flex(binding, doc_q=P) == 2                   # ids for both sides or neither
+    assert flex(binding, doc_kv=P) == 2
+    assert flex(binding, alibi=ctypes.c_void_p(18)) == 2  # misaligned slopes
+    assert flex(binding, Sk=128 * 1024 + 1) == 3          # longer than the flex kernel takes
+    assert flex(binding, B=0) == 0
+    assert flex(binding, Sq=0, softcap=3.0) == 0
+
+
+def _brute_block_states(keep):
+    Sq, Sk = keep.shape
+    out = np.zeros(((Sq + 63) // 64, (Sk + 63) // 64), np.uint8)
+    for qb in range(out.shape[0]):
+        for kb in range(out.shape[1]):
+            blk = keep[qb * 64:(qb + 1) * 64, kb * 64:(kb + 1) * 64]
+            out[qb, kb] = 2 if blk.all() else (1 if blk.any() else 0)
+    return out
+
+
+@pytest.mark.parametrize("Sq,Sk,causal,window,input_pos", [
+    (150, 200, 0, 0, 0), (150, 200, 1, 0, 0), (150, 200, 1, 16, 0), (130, 200, 1, 0, 50),
+    (64, 64, 1, 0, 0), (1, 300, 1, 7, 299)])
+def test_block_mask_document_matches_brute_force(binding, Sq, Sk, causal, window, input_pos):
+    import torch
+    from gqa_attention_flash_b200 import workloads as W
+    doc = W.document_ids(Sk, seed=Sq + Sk, min_len=1, max_len=70)
+    dq = doc[input_pos:input_pos + Sq].clone()
+    i = np.arange(Sq)[:, None] + input_pos
+    j = np.arange(Sk)[None, :]
+    keep = dq.numpy()[:, None] == doc.numpy()[None, :]
+    if causal:
+        keep &= j <= i
+    if window:
+        keep &= j > i - window
+    bm = binding.block_mask_document(Sq, Sk, dq, doc, causal, window, input_pos)
+    assert bm.dtype == torch.uint8 and tuple(bm.shape) == ((Sq + 63) // 64, (Sk + 63) // 64)
+    assert np.array_equal(bm.numpy(), _brute_block_states(keep))
+    bm2 = binding.block_mask_build(Sq, Sk, lambda q, kv: bool(keep[q - input_pos, kv]), input_pos)
+    assert np.array_equal(bm2.numpy(), _brute_block_states(keep))
+
+
+def test_block_mask_builder_validation(binding):
+    L = binding.lib
+    assert L.attn_block_mask_document(None, 4, 4, 0, 1, 0, P, P) == 1
+    assert L.attn_block_mask_document(P, 4, 4, 0, 0, 3, P, P) == 2   # window needs causal
+    assert L.attn_block_mask_document(P, -1, 4, 0, 1, 0, P, P) == 2
+    assert L.attn_block_mask_document(P, 0, 4, 0, 1, 0, None, None) == 0
