@@ -72,6 +72,8 @@ class Oracle:
         L.oracle_flex_fwd.argtypes = [_D, _D, _D, _D, _D] + [ctypes.c_int] * 6 + [
             ctypes.c_double, ctypes.c_int, ctypes.c_int, ctypes.c_int, _I, _I, _I, ctypes.c_int,
             ctypes.c_double, _D, _I, _I]
+        L.oracle_decode_paged.restype = ctypes.c_int
+        L.oracle_decode_paged.argtypes = [_D, _D, _D, _D, _D, _I, _I] + [ctypes.c_int] * 7
         L.oracle_decode.restype = ctypes.c_int
         L.oracle_decode.argtypes = [_D, _D, _D, _D, _D] + [ctypes.c_int] * 5 + [_I]
 
@@ -168,6 +170,30 @@ class Oracle:
                                     B, Hq, Hkv, S_cap, D, _iptr(ln))
         if rc != 0:
             raise ValueError("oracle_decode rejected its arguments")
+        return O, LSE
+
+
+    # -- vllm-mlx paged KV cache + decode_attention! ------------------------------------
+    def decode_paged(self, Q, K_cache, V_cache, block_tables, seq_lens):
+        """vllm-mlx paged KV cache decode: O (B,Hq,D) and LSE (B,Hq) float64.
+
+        Q (B, Hq, D); K_cache / V_cache (num_blocks, block_size, Hkv, D);
+        block_tables int (B, max_blocks); seq_lens int (B,).
+        """
+        Q, K, V = _f64(Q), _f64(K_cache), _f64(V_cache)
+        B, Hq, D = Q.shape
+        num_blocks, block_size, Hkv, Dk = K.shape
+        assert Dk == D and V.shape == K.shape
+        bt = np.ascontiguousarray(np.asarray(block_tables, dtype=np.int32))
+        assert bt.ndim == 2 and bt.shape[0] == B
+        ln = _i32(seq_lens)
+        O = np.empty((B, Hq, D), dtype=np.float64)
+        LSE = np.empty((B, Hq), dtype=np.float64)
+        rc = self.lib.oracle_decode_paged(_dptr(O), _dptr(LSE), _dptr(Q), _dptr(K), _dptr(V),
+                                          _iptr(bt), _iptr(ln), B, Hq, Hkv, num_blocks, block_size,
+                                          bt.shape[1], D)
+        if rc != 0:
+            raise ValueError("oracle_decode_paged rejected its arguments")
         return O, LSE
 
 

@@ -30,6 +30,12 @@
  *     precomputed `BlockMask` only tells a kernel which tiles to skip; when it
  *     agrees with the mask mod (as the page requires) it changes nothing in
  *     the result, so the oracle ignores it.
+ *   - vllm-mlx "attention" page, `MLXAttentionBackend.get_kv_cache_shape` and
+ *     `MLXAttentionMetadata` (seq_lens, block_tables): a paged KV cache of
+ *     shape (num_blocks, block_size, num_kv_heads, head_size); token j of
+ *     sequence b sits in block block_tables[b][j / block_size], slot
+ *     j % block_size.  Decoding from it is decode_attention! over the tokens
+ *     the block table gathers.
  *   - Tylo.jl "Primitives" page, entry `decode_attention!`: one query vector
  *     per head and sequence against the first lengths[b] cached keys.  The
  *     split into n_splits slices and their combine change only the rounding,
@@ -358,6 +364,86 @@ int oracle_decode(double *O, double *LSE, const double *Q, const double *K, cons
                 for (int d = 0; d < D; ++d) o[d] += p * Vb[j * D + d];
             }
             if (LSE) LSE[b * Hq + hq] = mx + log(l);
+        }
+        free(score);
+    }
+    return bad ? -1 : 0;
+}
+
+/*
+ * Paged decode (vllm-mlx "attention" page: KV cache shape (num_blocks,
+ * block_size, num_kv_heads, head_size), metadata seq_lens and block_tables)
+ * with the decode_attention! definition above: for sequence b and query head
+ * hq, key j < seq_lens[b] is row block_tables[b * max_blocks + j / block_size],
+ * slot j % block_size, KV head hq / (Hq / Hkv) of the cache; scale 1/sqrt(D).
+ *   Q (B, Hq, D); K_cache, V_cache (num_blocks, block_size, Hkv, D);
+ *   block_tables (B, max_blocks); O (B, Hq, D); LSE (B, Hq) or NULL.
+ * Returns 0, or -1 on bad arguments (a length above max_blocks * block_size or
+ * a referenced block outside 0 .. num_blocks-1).
+ */
+int oracle_decode_paged(double *O, double *LSE, const double *Q, const double *K_cache,
+                        const double *V_cache, const int *block_tables, const int *seq_lens,
+                        int B, int Hq, int Hkv, int num_blocks, int block_size, int max_blocks,
+                        int D) {
+    if (B < 0 || Hq <= 0 || Hkv <= 0 || num_blocks < 0 || block_size <= 0 || max_blocks < 0 ||
+        D <= 0 || seq_lens == NULL || (B > 0 && block_tables == NULL))
+        return -1;
+    if (Hq % Hkv != 0) return -1;
+    for (int b = 0; b < B; ++b) {
+        if (seq_lens[b] < 0 || (long)seq_lens[b] > (long)max_blocks * block_size) return -1;
+        for (long j = 0; j < seq_lens[b]; j += block_size) {
+            const int blk = block_tables[(long)b * max_blocks + j / block_size];
+            if (blk < 0 || blk >= num_blocks) return -1;
+        }
+    }
+    const int group = Hq / Hkv;
+    const double qk_scale = 1.0 / sqrt((double)D);
+    const long total = (long)B * Hq;
+    int bad = 0;
+
+#pragma omp parallel
+    {
+        long cap = (long)max_blocks * block_size;
+        double *score = (double *)malloc(sizeof(double) * (cap > 0 ? cap : 1));
+        if (score == NULL) {
+#pragma omp atomic write
+            bad = 1;
+        }
+#pragma omp for schedule(dynamic, 1)
+        for (long t = 0; t < total; ++t) {
+            if (score == NULL) continue;
+            const long hq = t % Hq;
+            const long b = t / Hq;
+            const long kvh = hq / group;
+            const int n = seq_lens[b];
+            const double *q = Q + (b * Hq + hq) * (long)D;
+            double *o = O + (b * Hq + hq) * (long)D;
+            for (int d = 0; d < D; ++d) o[d] = 0.0;
+            if (n == 0) {
+                if (LSE) LSE[b * Hq + hq] = -INFINITY;
+                continue;
+            }
+            double mx = -INFINITY;
+            for (long j = 0; j < n; ++j) {
+                const long blk = block_tables[b * max_blocks + j / block_size];
+                const double *kr = K_cache + ((blk * block_size + j % block_size) * Hkv + kvh) * D;
+                double dot = 0.0;
+                for (int d = 0; d < D; ++d) dot += q[d] * kr[d];
+                score[j] = qk_scale * dot;
+                if (score[j] > mx) mx = score[j];
+            }
+            double den = 0.0;
+            for (long j = 0; j < n; ++j) {
+                score[j] = exp(score[j] - mx);
+                den += score[j];
+            }
+            for (long j = 0; j < n; ++j) {
+                const long blk = block_tables[b * max_blocks + j / block_size];
+                const double *vr = V_cache + ((blk * block_size + j % block_size) * Hkv + kvh) * D;
+                const double w = score[j] / den;
+                for (int d = 0; d < D; ++d) o[d] += w * vr[d];
+            }
+            if (LSE) LSE[b * Hq + hq] = mx + log(den);
         }
         free(score);
     }

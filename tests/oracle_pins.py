@@ -422,6 +422,66 @@ def pin_flex_document_blocks(orc):
             a += n
 
 
+# --------------------------------------------------------------------------------------
+# vllm-mlx "attention" page: paged KV cache (num_blocks, block_size, num_kv_heads,
+# head_size) with block tables, decoded with decode_attention!
+# --------------------------------------------------------------------------------------
+
+def _scatter_paged(K, V, lengths, block_size, rng, extra_blocks=3):
+    """Scatter contiguous caches (B, Hkv, S_cap, D) into a shuffled block pool."""
+    B, Hkv, S_cap, D = K.shape
+    max_blocks = -(-S_cap // block_size)
+    n_blocks = B * max_blocks + extra_blocks
+    perm = rng.permutation(n_blocks)[:B * max_blocks].reshape(B, max_blocks)
+    Kc = rng.standard_normal((n_blocks, block_size, Hkv, D))
+    Vc = rng.standard_normal((n_blocks, block_size, Hkv, D))
+    for b in range(B):
+        for lb in range(max_blocks):
+            j0, j1 = lb * block_size, min((lb + 1) * block_size, S_cap)
+            Kc[perm[b, lb], :j1 - j0] = K[b, :, j0:j1].transpose(1, 0, 2)
+            Vc[perm[b, lb], :j1 - j0] = V[b, :, j0:j1].transpose(1, 0, 2)
+    return Kc, Vc, perm.astype(np.int32)
+
+
+def pin_paged_equals_contiguous(orc):
+    """A cache scattered into shuffled blocks and read back through the block table
+    decodes exactly like the contiguous cache (decode_attention!), for several
+    block sizes, with GQA, and for lengths 0, 1, block edges and the capacity."""
+    rng = _rng(31)
+    B, Hq, Hkv, S_cap, D = 5, 6, 2, 37, 8
+    Q = rng.standard_normal((B, Hq, D))
+    K, V = rng.standard_normal((B, Hkv, S_cap, D)), rng.standard_normal((B, Hkv, S_cap, D))
+    lengths = np.array([0, 1, 16, 33, 37], dtype=np.int32)
+    O0, L0 = orc.decode(Q, K, V, lengths)
+    for bs in (1, 4, 16, 64):
+        Kc, Vc, bt = _scatter_paged(K, V, lengths, bs, rng)
+        O1, L1 = orc.decode_paged(Q, Kc, Vc, bt, lengths)
+        assert np.max(np.abs(O1 - O0)) < 1e-12, bs
+        assert np.array_equal(np.isneginf(L1), np.isneginf(L0))
+        fin = ~np.isneginf(L0)
+        assert np.max(np.abs(L1[fin] - L0[fin])) < 1e-12, bs
+
+
+def pin_paged_reads_only_listed_slots(orc):
+    """Blocks the table does not reach, and slots past a sequence's length, may hold
+    anything (here NaN): the result stays finite and equal."""
+    rng = _rng(32)
+    B, Hq, Hkv, S_cap, D, bs = 3, 4, 4, 20, 8, 8
+    Q = rng.standard_normal((B, Hq, D))
+    K, V = rng.standard_normal((B, Hkv, S_cap, D)), rng.standard_normal((B, Hkv, S_cap, D))
+    lengths = np.array([5, 20, 9], dtype=np.int32)
+    Kc, Vc, bt = _scatter_paged(K, V, lengths, bs, rng)
+    O0, L0 = orc.decode_paged(Q, Kc, Vc, bt, lengths)
+    used = np.zeros(Kc.shape[:2], dtype=bool)
+    for b in range(B):
+        for j in range(lengths[b]):
+            used[bt[b, j // bs], j % bs] = True
+    Kc[~used] = np.nan
+    Vc[~used] = np.nan
+    O1, L1 = orc.decode_paged(Q, Kc, Vc, bt, lengths)
+    assert np.all(np.isfinite(O1)) and np.array_equal(O1, O0) and np.array_equal(L1, L0)
+
+
 PINS = [
     pin_causal_mask_shape_and_rows,
     pin_sliding_window_rows,
@@ -441,4 +501,6 @@ PINS = [
     pin_flex_softcap_limits,
     pin_flex_alibi_geometric,
     pin_flex_document_blocks,
+    pin_paged_equals_contiguous,
+    pin_paged_reads_only_listed_slots,
 ]

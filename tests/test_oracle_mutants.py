@@ -51,6 +51,18 @@ MUTANTS = {
     "flex_gqa_modulo": ("const long kv_head = hq / group;", "const long kv_head = hq % Hkv;"),
     "flex_lse_missing_max": ("if (LSE) LSE[row_id] = mx + log(lsum);", "if (LSE) LSE[row_id] = log(lsum);"),
     "flex_not_normalised": ("const double pj = score[j] / lsum;", "const double pj = score[j];"),
+    "paged_slot_by_block": ("const double *kr = K_cache + ((blk * block_size + j % block_size) * Hkv + kvh) * D;",
+                            "const double *kr = K_cache + ((blk * block_size + j / block_size) * Hkv + kvh) * D;"),
+    "paged_table_ignored": ("const long blk = block_tables[b * max_blocks + j / block_size];\n"
+                            "                const double *kr",
+                            "const long blk = b * max_blocks + j / block_size;\n"
+                            "                const double *kr"),
+    "paged_head_stride": ("const double *vr = V_cache + ((blk * block_size + j % block_size) * Hkv + kvh) * D;",
+                          "const double *vr = V_cache + ((blk * block_size + j % block_size) + kvh) * D;"),
+    "paged_v_from_k": ("const double *vr = V_cache +", "const double *vr = K_cache +"),
+    "paged_scale": ("const double qk_scale = 1.0 / sqrt((double)D);", "const double qk_scale = 1.0 / (double)D;"),
+    "paged_lse_missing_max": ("if (LSE) LSE[b * Hq + hq] = mx + log(den);",
+                              "if (LSE) LSE[b * Hq + hq] = log(den);"),
 }
 
 
