@@ -399,6 +399,49 @@ def time_flex(dev, steps, warmup, peak):
     return out
 
 
+def time_paged(step, steps, warmup, peak):
+    """Paged-KV decode row: the step's decode sequences scattered into a shuffled
+    pool of 16-token blocks (block tables), device-resident; CUDA events around
+    each launch; GB/s on the same algorithmic bytes as the contiguous decode."""
+    from gqa_attention_flash_b200 import binding
+    w = W.PAGED_DECODE
+    d = step.dw
+    lengths = step.lengths_host.tolist()
+    tables, num_blocks = W.paged_layout(lengths, w.block_size, w.spare, w.seed)
+    shape = (num_blocks, w.block_size, d.Hkv, d.D)
+    Kp = torch.zeros(shape, dtype=torch.bfloat16, device=step.dev)
+    Vp = torch.zeros(shape, dtype=torch.bfloat16, device=step.dev)
+    W.fill_paged_cache(Kp, Vp, tables, lambda b: (step.Kc[b, :, :lengths[b]],
+                                                  step.Vc[b, :, :lengths[b]]))
+    tdev = tables.to(step.dev)
+    O = torch.empty_like(step.dQ)
+
+    def run():
+        binding.attn_decode_paged(O, step.dQ, Kp, Vp, tdev, step.lengths, d.n_splits)
+    for _ in range(warmup):
+        run()
+    torch.cuda.synchronize()
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+          for _ in range(steps)]
+    for e0, e1 in ev:
+        e0.record()
+        run()
+        e1.record()
+    torch.cuda.synchronize()
+    st = binding.last_device_status()
+    if st != 0:
+        raise RuntimeError(f"paged decode device status: {binding.status_string(st)}")
+    ms = sum(a.elapsed_time(b) for a, b in ev) / steps
+    gbs = step.decode_bytes / (ms * 1e-3) / 1e9
+    del Kp, Vp
+    torch.cuda.empty_cache()
+    return {"workload": w.name, "value": gbs, "unit": "GB/s", "ms_per_launch": ms,
+            "bytes_per_launch": step.decode_bytes, "launches": steps, "num_blocks": num_blocks,
+            "roofline": {"bound": "hbm", "achieved": gbs, "peak": peak, "unit": "GB/s",
+                         "frac": gbs / peak,
+                         "kernel": "decode_split_kernel<128, paged> + decode_combine_kernel<128>"}}
+
+
 def cpu_model():
     try:
         with open("/proc/cpuinfo") as f:
@@ -484,7 +527,9 @@ def main(argv=None):
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-flex", action="store_true",
                     help="skip the flex_attention! measurements (reported apart from the step)")
-    ap.add_argument("--only", choices=["prefill", "decode", "flex"], default=None,
+    ap.add_argument("--no-paged", action="store_true",
+                    help="skip the paged-KV decode measurement (reported apart from the step)")
+    ap.add_argument("--only", choices=["prefill", "decode", "flex", "paged"], default=None,
                     help="profiling: run one half of the step, or only the flex_attention! "
                          "workloads (no reported number)")
     ap.add_argument("--decode-batch", type=int, default=None,
@@ -507,6 +552,12 @@ def main(argv=None):
         barrier = lambda: None  # noqa: E731
     dev = torch.device("cuda", local_rank)
     torch.cuda.set_device(dev)
+    if args.only == "paged":
+        peaks, _ = load_peaks()
+        pstep = Step(dev, "decode", args.decode_batch)
+        res = time_paged(pstep, args.steps, args.warmup, peaks["hbm_gbs"])
+        print(json.dumps({"profiling_run": True, "paged_ms": res["ms_per_launch"]}), flush=True)
+        return 0
     if args.only == "flex":
         peaks, _ = load_peaks()
         res = time_flex(dev, args.steps, args.warmup, peaks["bf16_tflops"])
@@ -580,6 +631,8 @@ def main(argv=None):
         line["cpu_baseline"] = cpu_baseline(step.host_prefill, step.dQ_host, step.lengths_host)
     if not args.no_flex:
         line["flex"] = time_flex(dev, min(K, 50), args.warmup, peaks["bf16_tflops"])
+    if not args.no_paged and step.do_decode:
+        line["paged_decode"] = time_paged(step, min(K, 100), args.warmup, peaks["hbm_gbs"])
     print(json.dumps(line), flush=True)
     if world > 1:
         dist.destroy_process_group()

@@ -44,6 +44,8 @@ lib.attn_block_mask_document.restype = _i
 lib.attn_block_mask_document.argtypes = [_p, _i, _i, _i, _i, _i, _p, _p]
 lib.attn_decode.restype = _i
 lib.attn_decode.argtypes = [_p, _p, _p, _p, _p, _i, _p] + [_i] * 5
+lib.attn_decode_paged.restype = _i
+lib.attn_decode_paged.argtypes = [_p, _p, _p, _p, _p, _p, _i, _p] + [_i] * 7
 lib.attn_decode_noalloc.restype = _i
 lib.attn_decode_noalloc.argtypes = [_p, _p, _p, _p, _p, _i, _p] + [_i] * 5
 lib.attn_status_string.restype = ctypes.c_char_p
@@ -148,6 +150,17 @@ def attn_decode(O, Q, K, V, lengths, n_splits=8, stream=None):
     rc = lib.attn_decode(_ptr(O), _ptr(Q), _ptr(K), _ptr(V), _ptr(lengths), int(n_splits),
                          _stream(stream), B, Hq, Hkv, S_cap, D)
     _check(rc, "attn_decode")
+
+
+def attn_decode_paged(O, Q, K_cache, V_cache, block_tables, seq_lens, n_splits=8, stream=None):
+    """Decode from a paged cache: Q (B,Hq,D); K/V caches (num_blocks, block_size, Hkv, D);
+    block_tables int32 (B, max_blocks); seq_lens int32 (B,); O (B,Hq,D) filled in place."""
+    B, Hq, D = Q.shape
+    num_blocks, block_size, Hkv, _ = K_cache.shape
+    rc = lib.attn_decode_paged(_ptr(O), _ptr(Q), _ptr(K_cache), _ptr(V_cache), _ptr(block_tables),
+                               _ptr(seq_lens), int(n_splits), _stream(stream), B, Hq, Hkv,
+                               num_blocks, block_size, int(block_tables.shape[1]), D)
+    _check(rc, "attn_decode_paged")
 
 
 def attn_decode_noalloc(O, Q, K, V, lengths, n_splits=8, stream=None):

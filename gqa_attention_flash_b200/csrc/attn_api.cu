@@ -74,6 +74,20 @@ attn_status_t make_tmap_bf16_3d(CUtensorMap *map, const void *base, uint64_t D, 
     return r == CUDA_SUCCESS ? ATTN_OK : ATTN_ERR_INVALID;
 }
 
+attn_status_t make_tmap_bf16_paged(CUtensorMap *map, const void *base, uint64_t D, uint64_t heads,
+                                   uint64_t rows, uint32_t box_rows) {
+    EncodeTiledFn fn = encode_fn();
+    if (!fn) return ATTN_ERR_CUDA;
+    const cuuint64_t dims[3] = {D, heads, rows > 0 ? rows : 1};
+    const cuuint64_t strides[2] = {D * 2, D * 2 * heads};
+    const cuuint32_t box[3] = {64, 1, box_rows};
+    const cuuint32_t estr[3] = {1, 1, 1};
+    CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void *>(base), dims,
+                    strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                    CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS ? ATTN_OK : ATTN_ERR_INVALID;
+}
+
 namespace {
 
 __global__ void wait_probe_kernel(uint64_t limit_ns) {
@@ -257,6 +271,52 @@ attn_status_t attn_decode(void *O, const void *Q, const void *K, const void *V,
     a.S_cap = S_cap;
     a.D = D;
     a.workspace = static_cast<float *>(ws);
+    attn_status_t st = launch_decode(a, s);
+    if (cudaFreeAsync(ws, s) != cudaSuccess && st == ATTN_OK) st = ATTN_ERR_CUDA;
+    return st;
+}
+
+attn_status_t attn_decode_paged(void *O, const void *Q, const void *K_cache, const void *V_cache,
+                                const int32_t *block_tables, const int32_t *seq_lens, int n_splits,
+                                void *stream, int B, int Hq, int Hkv, int num_blocks,
+                                int block_size, int max_blocks_per_seq, int D) {
+    if (B < 0 || Hq < 1 || Hkv < 1 || num_blocks < 1 || max_blocks_per_seq < 0 || n_splits < 1 ||
+        n_splits > 64)
+        return ATTN_ERR_INVALID;
+    if (block_size < 8 || block_size > 65536 || (block_size & (block_size - 1)) != 0)
+        return ATTN_ERR_INVALID;
+    if (Hq % Hkv != 0 || Hq / Hkv > 16) return ATTN_ERR_INVALID;
+    if (D != 64 && D != 128) return ATTN_ERR_UNSUPPORTED;
+    if ((long long)num_blocks * block_size > 0x7fffffffll ||
+        (long long)max_blocks_per_seq * block_size > 0x7fffffffll)
+        return ATTN_ERR_INVALID;
+    if (B == 0) return ATTN_OK;
+    if (!O || !Q || !K_cache || !V_cache || !seq_lens || (max_blocks_per_seq > 0 && !block_tables))
+        return ATTN_ERR_NULL;
+    if (!aligned16(O) || !aligned16(Q) || !aligned16(K_cache) || !aligned16(V_cache) ||
+        ((reinterpret_cast<uintptr_t>(seq_lens) | reinterpret_cast<uintptr_t>(block_tables)) & 3u))
+        return ATTN_ERR_INVALID;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    const size_t bytes = decode_workspace_floats(B, Hq, n_splits, D) * sizeof(float);
+    void *ws = nullptr;
+    if (cudaMallocAsync(&ws, bytes, s) != cudaSuccess) return ATTN_ERR_CUDA;
+    DecodeArgs a;
+    a.O = O;
+    a.Q = Q;
+    a.K = K_cache;
+    a.V = V_cache;
+    a.lengths = seq_lens;
+    a.n_splits = n_splits;
+    a.B = B;
+    a.Hq = Hq;
+    a.Hkv = Hkv;
+    a.S_cap = max_blocks_per_seq * block_size;
+    a.D = D;
+    a.workspace = static_cast<float *>(ws);
+    a.block_tables = block_tables;
+    a.num_blocks = num_blocks;
+    a.block_size = block_size;
+    a.max_blocks = max_blocks_per_seq;
     attn_status_t st = launch_decode(a, s);
     if (cudaFreeAsync(ws, s) != cudaSuccess && st == ATTN_OK) st = ATTN_ERR_CUDA;
     return st;

@@ -17,6 +17,11 @@
 // the slice's normalised partial output and log-sum-exp are written to the
 // workspace.
 //
+// Paged variant (vllm-mlx "attention" page: KV cache of shape (num_blocks,
+// block_size, num_kv_heads, head_size), metadata seq_lens and block_tables):
+// the same kernels, with each 64-key tile gathered by TMA from the blocks the
+// sequence's block table names, block_size (or 64) rows of one head per copy.
+//
 // Kernel 2 (combine): one warp per (sequence, query head) merges the slices:
 // LSE = log sum_s exp(lse_s), O = sum_s exp(lse_s - LSE) o_s; empty slices
 // (lse = -inf) weigh nothing, and a sequence with no valid key gets O = 0.
@@ -60,6 +65,9 @@ struct DecParams {
     float scale_log2;
     uint64_t wait_limit_ns;
     int *status;  // device status word
+    // paged cache only
+    const int32_t *block_tables;  // (B, max_blocks)
+    int max_blocks, block_shift, num_blocks, box_rows;
 };
 
 __device__ __forceinline__ float neg_inf() { return __int_as_float(0xff800000); }
@@ -70,7 +78,7 @@ __device__ __forceinline__ uint32_t swz(int row, int chunk) {
     return (chunk >> 3) * (TN * 128) + row * 128 + (((chunk & 7) ^ (row & 7)) << 4);
 }
 
-template <int D>
+template <int D, bool kPaged>
 __global__ void __launch_bounds__(kDecThreads)
     decode_split_kernel(const __grid_constant__ CUtensorMap tmK,
                         const __grid_constant__ CUtensorMap tmV, const DecParams p) {
@@ -134,12 +142,35 @@ __global__ void __launch_bounds__(kDecThreads)
                     !mbar_wait(empty(st), (use - 1) & 1, abort_flag, p.wait_limit_ns, p.status))
                     break;
                 const int row = (t_begin + it) * TN;
-                mbar_arrive_expect_tx(full(st), 2 * C::TILE);
-                for (int c = 0; c < C::NBOX; ++c) {
-                    tma_load_3d(sbase + C::OFF_K + st * C::TILE + c * C::BOX, &tmK, full(st),
-                                c * 64, row, b * p.Hkv + hkv);
-                    tma_load_3d(sbase + C::OFF_V + st * C::TILE + c * C::BOX, &tmV, full(st),
-                                c * 64, row, b * p.Hkv + hkv);
+                if constexpr (!kPaged) {
+                    mbar_arrive_expect_tx(full(st), 2 * C::TILE);
+                    for (int c = 0; c < C::NBOX; ++c) {
+                        tma_load_3d(sbase + C::OFF_K + st * C::TILE + c * C::BOX, &tmK, full(st),
+                                    c * 64, row, b * p.Hkv + hkv);
+                        tma_load_3d(sbase + C::OFF_V + st * C::TILE + c * C::BOX, &tmV, full(st),
+                                    c * 64, row, b * p.Hkv + hkv);
+                    }
+                } else {
+                    // Gather the tile's valid keys chunk by chunk: key j of the sequence
+                    // is cache row block_tables[b][j / block_size] * block_size +
+                    // j % block_size.  Chunks past the length are not loaded; the
+                    // consumers mask those keys and zero those V rows.
+                    const int br = p.box_rows;
+                    const int n_chunks = (min(TN, len - row) + br - 1) / br;
+                    mbar_arrive_expect_tx(full(st), 2 * n_chunks * br * 128 * C::NBOX);
+                    const int32_t *bt = p.block_tables + (long long)b * p.max_blocks;
+                    for (int k = 0; k < n_chunks; ++k) {
+                        const int j = row + k * br;
+                        const int blk = bt[j >> p.block_shift];
+                        if (blk < 0 || blk >= p.num_blocks) record_status(p.status, ATTN_ERR_DEVICE_BOUNDS);
+                        // an out-of-range block reads as zeros (outside the tensor map)
+                        const int prow = blk * (1 << p.block_shift) + (j & ((1 << p.block_shift) - 1));
+                        for (int c = 0; c < C::NBOX; ++c) {
+                            const uint32_t off = st * C::TILE + c * C::BOX + k * br * 128;
+                            tma_load_3d(sbase + C::OFF_K + off, &tmK, full(st), c * 64, hkv, prow);
+                            tma_load_3d(sbase + C::OFF_V + off, &tmV, full(st), c * 64, hkv, prow);
+                        }
+                    }
                 }
             }
         }
@@ -357,18 +388,25 @@ __global__ void __launch_bounds__(128)
     }
 }
 
-template <int D>
+template <int D, bool kPaged>
 attn_status_t launch_decode_d(const DecodeArgs &a, cudaStream_t stream) {
     using C = DecCfg<D>;
     CUtensorMap tk, tv;
     attn_status_t st;
-    if ((st = make_tmap_bf16_3d(&tk, a.K, D, a.S_cap, (uint64_t)a.B * a.Hkv, TN)) != ATTN_OK)
-        return st;
-    if ((st = make_tmap_bf16_3d(&tv, a.V, D, a.S_cap, (uint64_t)a.B * a.Hkv, TN)) != ATTN_OK)
-        return st;
+    const uint32_t box_rows = kPaged ? static_cast<uint32_t>(min(a.block_size, TN)) : TN;
+    if constexpr (kPaged) {
+        const uint64_t rows = (uint64_t)a.num_blocks * a.block_size;
+        if ((st = make_tmap_bf16_paged(&tk, a.K, D, a.Hkv, rows, box_rows)) != ATTN_OK) return st;
+        if ((st = make_tmap_bf16_paged(&tv, a.V, D, a.Hkv, rows, box_rows)) != ATTN_OK) return st;
+    } else {
+        if ((st = make_tmap_bf16_3d(&tk, a.K, D, a.S_cap, (uint64_t)a.B * a.Hkv, TN)) != ATTN_OK)
+            return st;
+        if ((st = make_tmap_bf16_3d(&tv, a.V, D, a.S_cap, (uint64_t)a.B * a.Hkv, TN)) != ATTN_OK)
+            return st;
+    }
     static bool configured = false;
     if (!configured) {
-        if (cudaFuncSetAttribute(decode_split_kernel<D>,
+        if (cudaFuncSetAttribute(decode_split_kernel<D, kPaged>,
                                  cudaFuncAttributeMaxDynamicSharedMemorySize,
                                  C::SMEM_BYTES) != cudaSuccess)
             return ATTN_ERR_CUDA;
@@ -388,8 +426,14 @@ attn_status_t launch_decode_d(const DecodeArgs &a, cudaStream_t stream) {
     p.wait_limit_ns = kWaitLimitNs;
     p.status = device_status_word();
     if (!p.status) return ATTN_ERR_CUDA;
+    p.block_tables = a.block_tables;
+    p.max_blocks = a.max_blocks;
+    p.num_blocks = a.num_blocks;
+    p.box_rows = static_cast<int>(box_rows);
+    p.block_shift = 0;
+    while (kPaged && (1 << p.block_shift) < a.block_size) ++p.block_shift;
     dim3 grid(a.n_splits, a.Hkv, a.B);
-    decode_split_kernel<D><<<grid, kDecThreads, C::SMEM_BYTES, stream>>>(tk, tv, p);
+    decode_split_kernel<D, kPaged><<<grid, kDecThreads, C::SMEM_BYTES, stream>>>(tk, tv, p);
     if (cudaGetLastError() != cudaSuccess) return ATTN_ERR_CUDA;
     const int BH = a.B * a.Hq;
     decode_combine_kernel<D><<<(BH + 3) / 4, 128, 0, stream>>>(static_cast<__nv_bfloat16 *>(a.O),
@@ -405,8 +449,13 @@ size_t decode_workspace_floats(int B, int Hq, int n_splits, int D) {
 
 attn_status_t launch_decode(const DecodeArgs &a, cudaStream_t stream) {
     if (a.B == 0) return ATTN_OK;
-    if (a.D == 128) return launch_decode_d<128>(a, stream);
-    if (a.D == 64) return launch_decode_d<64>(a, stream);
+    if (a.block_tables) {
+        if (a.D == 128) return launch_decode_d<128, true>(a, stream);
+        if (a.D == 64) return launch_decode_d<64, true>(a, stream);
+        return ATTN_ERR_UNSUPPORTED;
+    }
+    if (a.D == 128) return launch_decode_d<128, false>(a, stream);
+    if (a.D == 64) return launch_decode_d<64, false>(a, stream);
     return ATTN_ERR_UNSUPPORTED;
 }
 

@@ -14,6 +14,12 @@ namespace gqa {
 attn_status_t make_tmap_bf16_3d(CUtensorMap *map, const void *base, uint64_t D, uint64_t rows,
                                 uint64_t outer, uint32_t box_rows);
 
+// Encode a 3-D bf16 tensor map over a paged cache viewed as (rows, heads, D)
+// row-major, with a (64, 1, box_rows) box and 128-byte swizzle: one box is
+// box_rows consecutive cache rows of one head, 64 columns wide.
+attn_status_t make_tmap_bf16_paged(CUtensorMap *map, const void *base, uint64_t D, uint64_t heads,
+                                   uint64_t rows, uint32_t box_rows);
+
 struct FwdArgs {
     void *O;
     const void *Q, *K, *V;
@@ -40,7 +46,11 @@ struct DecodeArgs {
     const int32_t *lengths;
     int n_splits;
     int B, Hq, Hkv, S_cap, D;
-    float *workspace;  // B * Hq * n_splits * (D + 1) floats
+    float *workspace;  // B * Hq * n_splits * (D + 4) floats
+    // paged KV cache (block_tables != nullptr): K/V are (num_blocks, block_size,
+    // Hkv, D) and S_cap = max_blocks * block_size
+    const int32_t *block_tables = nullptr;
+    int num_blocks = 0, block_size = 0, max_blocks = 0;
 };
 
 // Device address of the status word on the current device (looked up once per

@@ -250,6 +250,71 @@ def fill_decode_cache(w: DecodeWorkload, lengths, K_cache, V_cache, fill: float 
         V_cache[b, :, :n].copy_(Vb, non_blocking=False)
 
 
+@dataclass(frozen=True)
+class PagedDecodeWorkload:
+    """Decode from a paged KV cache (num_blocks, block_size, Hkv, D): the same
+    queries, lengths and per-sequence K/V as ``base``, scattered into a pool of
+    blocks in a seeded random order (plus ``spare`` unused blocks)."""
+    name: str
+    base: DecodeWorkload
+    block_size: int
+    spare: int = 64
+    seed: int = 7
+
+
+PAGED_DECODE = PagedDecodeWorkload("paged split-KV decode B64 Hq32 Hkv8 D128 block 16, "
+                                   "lengths 1024..32768, n_splits 8", DECODE, 16)
+
+
+def paged_layout(lengths, block_size: int, spare: int, seed: int):
+    """(block_tables int32 (B, max_blocks), num_blocks): every sequence's logical
+    blocks mapped to distinct physical blocks in a random order; table entries past
+    a sequence's last block are -1."""
+    n_blk = [(int(n) + block_size - 1) // block_size for n in lengths]
+    max_blocks = max(1, max(n_blk) if n_blk else 1)
+    num_blocks = sum(n_blk) + spare
+    g = torch.Generator(device="cpu").manual_seed(seed)
+    perm = torch.randperm(num_blocks, generator=g).to(torch.int32)
+    tables = torch.full((len(n_blk), max_blocks), -1, dtype=torch.int32)
+    pos = 0
+    for b, n in enumerate(n_blk):
+        tables[b, :n] = perm[pos:pos + n]
+        pos += n
+    return tables, num_blocks
+
+
+def fill_paged_cache(K_pool, V_pool, tables, seq_kv):
+    """Scatter per-sequence (Hkv, length, D) K/V (``seq_kv(b)`` returns them) into the
+    block pools (num_blocks, block_size, Hkv, D) along the block tables."""
+    bs = K_pool.shape[1]
+    for b in range(tables.shape[0]):
+        Kb, Vb = seq_kv(b)
+        n = Kb.shape[1]
+        nb = (n + bs - 1) // bs
+        if nb == 0:
+            continue
+        idx = tables[b, :nb].to(torch.long).to(K_pool.device)
+        for src, pool in ((Kb, K_pool), (Vb, V_pool)):
+            pad = torch.zeros(src.shape[0], nb * bs, src.shape[2], dtype=src.dtype,
+                              device=src.device)
+            pad[:, :n] = src
+            blocks = pad.reshape(src.shape[0], nb, bs, src.shape[2]).permute(1, 2, 0, 3)
+            pool.index_copy_(0, idx, blocks.contiguous().to(pool.device))
+
+
+def make_paged_decode(w: PagedDecodeWorkload, device="cpu"):
+    """Q (B,Hq,D), K/V pools, block tables and seq_lens of a paged decode workload."""
+    d = w.base
+    Q, lengths = decode_query_and_lengths(d)
+    tables, num_blocks = paged_layout(lengths.tolist(), w.block_size, w.spare, w.seed)
+    shape = (num_blocks, w.block_size, d.Hkv, d.D)
+    K_pool = torch.zeros(shape, dtype=torch.bfloat16, device=device)
+    V_pool = torch.zeros(shape, dtype=torch.bfloat16, device=device)
+    fill_paged_cache(K_pool, V_pool, tables,
+                     lambda b: decode_sequence_kv(d, b, int(lengths[b])))
+    return Q, K_pool, V_pool, tables, lengths
+
+
 def decode_bytes(w: DecodeWorkload, lengths) -> int:
     """Algorithmic bytes of one decode: the valid K/V prefix plus Q and O."""
     kv = 2 * w.Hkv * w.D * 2 * int(sum(int(x) for x in lengths))

@@ -184,6 +184,30 @@ attn_status_t attn_decode(void *O, const void *Q, const void *K, const void *V,
                           int B, int Hq, int Hkv, int S_cap, int D);
 
 /*
+ * attn_decode_paged -- attn_decode over a paged KV cache (vllm-mlx
+ * "attention" page: MLXAttentionBackend.get_kv_cache_shape gives the cache
+ * shape (num_blocks, block_size, num_kv_heads, head_size); MLXAttentionMetadata
+ * carries seq_lens and block_tables).
+ *
+ *   O       [out] bf16 (B, Hq, D)
+ *   Q       [in]  bf16 (B, Hq, D), one new token per sequence
+ *   K_cache, V_cache [in] bf16 (num_blocks, block_size, Hkv, D)
+ *   block_tables [in] int32 (B, max_blocks_per_seq) device array: key j of
+ *           sequence b is row j % block_size of block block_tables[b][j /
+ *           block_size].  Entries past a sequence's last block are not read.
+ *   seq_lens [in] int32 (B,) device array: keys 0 .. seq_lens[b]-1 attend.
+ *           Values above max_blocks_per_seq * block_size are clamped and
+ *           flagged ATTN_ERR_DEVICE_BOUNDS, as is a block index outside
+ *           0 .. num_blocks-1 (that block then reads as zeros).
+ *   n_splits, scale (1/sqrt(D)), GQA rule, workspace and errors as attn_decode.
+ *   block_size: a power of two >= 8.
+ */
+attn_status_t attn_decode_paged(void *O, const void *Q, const void *K_cache, const void *V_cache,
+                                const int32_t *block_tables, const int32_t *seq_lens, int n_splits,
+                                void *stream, int B, int Hq, int Hkv, int num_blocks,
+                                int block_size, int max_blocks_per_seq, int D);
+
+/*
  * attn_decode_noalloc -- attn_decode for callers that cannot allocate device
  * memory.  The pages have no counterpart: it is attn_decode with a different
  * home for the per-slice workspace.

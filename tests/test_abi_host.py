@@ -163,3 +163,37 @@ def test_block_mask_builder_validation(binding):
     assert L.attn_block_mask_document(P, 4, 4, 0, 0, 3, P, P) == 2   # window needs causal
     assert L.attn_block_mask_document(P, -1, 4, 0, 1, 0, P, P) == 2
     assert L.attn_block_mask_document(P, 0, 4, 0, 1, 0, None, None) == 0
+
+
+def test_decode_paged_host_validation(binding):
+    L = binding.lib
+
+    def dec(**kw):
+        a = dict(O=P, Q=P, K=P, V=P, bt=P, lens=P, n_splits=8, B=2, Hq=8, Hkv=2, num_blocks=10,
+                 block_size=16, max_blocks=4, D=128)
+        a.update(kw)
+        return L.attn_decode_paged(a["O"], a["Q"], a["K"], a["V"], a["bt"], a["lens"],
+                                   a["n_splits"], None, a["B"], a["Hq"], a["Hkv"],
+                                   a["num_blocks"], a["block_size"], a["max_blocks"], a["D"])
+    assert dec(block_size=12) == 2      # not a power of two
+    assert dec(block_size=4) == 2       # below 8
+    assert dec(num_blocks=0) == 2
+    assert dec(n_splits=0) == 2
+    assert dec(Hq=6, Hkv=4) == 2
+    assert dec(D=96) == 3
+    assert dec(bt=None) == 1
+    assert dec(lens=None) == 1
+    assert dec(K=ctypes.c_void_p(24)) == 2
+    assert dec(B=0) == 0
+
+
+def test_paged_layout_helper():
+    from gqa_attention_flash_b200 import workloads as W
+    lengths = [5, 17, 0, 32, 48]
+    tables, n = W.paged_layout(lengths, 16, 3, 1)
+    used = tables[tables >= 0]
+    assert n == 1 + 2 + 0 + 2 + 3 + 3
+    assert len(set(used.tolist())) == used.numel() and int(used.max()) < n
+    for b, ln in enumerate(lengths):
+        nb = (ln + 15) // 16
+        assert bool((tables[b, :nb] >= 0).all()) and bool((tables[b, nb:] == -1).all())
