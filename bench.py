@@ -45,6 +45,10 @@ KERNEL_SOURCES = {
                         "gqa_attention_flash_b200/csrc/sm100_ptx.cuh"],
     "decode_split_kernel": ["gqa_attention_flash_b200/csrc/attn_decode.cu",
                             "gqa_attention_flash_b200/csrc/sm100_ptx.cuh"],
+    "attn_fwd_kernel_flex_doc_softcap": ["gqa_attention_flash_b200/csrc/attn_fwd.cu",
+                                         "gqa_attention_flash_b200/csrc/sm100_ptx.cuh"],
+    "decode_split_kernel_paged": ["gqa_attention_flash_b200/csrc/attn_decode.cu",
+                                  "gqa_attention_flash_b200/csrc/sm100_ptx.cuh"],
 }
 
 
@@ -393,6 +397,8 @@ def time_flex(dev, steps, warmup, peak):
                     "flops_per_launch": flops, "launches": steps,
                     "roofline": {"bound": "tensor", "achieved": tf, "peak": peak,
                                  "unit": "TFLOP/s", "frac": tf / peak,
+                                 "traffic": ncu_traffic("attn_fwd_kernel_flex_" + key)
+                                 if "attn_fwd_kernel_flex_" + key in KERNEL_SOURCES else None,
                                  "kernel": "attn_fwd_kernel<128, flex>"}}
         del Qd, Kd, Vd, O, LSE
         torch.cuda.empty_cache()
@@ -438,7 +444,7 @@ def time_paged(step, steps, warmup, peak):
     return {"workload": w.name, "value": gbs, "unit": "GB/s", "ms_per_launch": ms,
             "bytes_per_launch": step.decode_bytes, "launches": steps, "num_blocks": num_blocks,
             "roofline": {"bound": "hbm", "achieved": gbs, "peak": peak, "unit": "GB/s",
-                         "frac": gbs / peak,
+                         "frac": gbs / peak, "traffic": ncu_traffic("decode_split_kernel_paged"),
                          "kernel": "decode_split_kernel<128, paged> + decode_combine_kernel<128>"}}
 
 
