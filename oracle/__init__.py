@@ -71,7 +71,13 @@ class Oracle:
         L.oracle_flex_fwd.restype = ctypes.c_int
         L.oracle_flex_fwd.argtypes = [_D, _D, _D, _D, _D] + [ctypes.c_int] * 6 + [
             ctypes.c_double, ctypes.c_int, ctypes.c_int, ctypes.c_int, _I, _I, _I, ctypes.c_int,
-            ctypes.c_double, _D, _I, _I]
+            ctypes.c_double, _D, _I, _I, ctypes.c_void_p]
+        L.oracle_rbs_block_scores.restype = ctypes.c_int
+        L.oracle_rbs_block_scores.argtypes = [_D, _D, _D, _D] + [ctypes.c_int] * 6
+        L.oracle_rbs_block_mask.restype = ctypes.c_int
+        L.oracle_rbs_block_mask.argtypes = [ctypes.c_void_p, _D, _D, ctypes.c_long, ctypes.c_int,
+                                            ctypes.c_int, ctypes.c_double, ctypes.c_double,
+                                            ctypes.c_int]
         L.oracle_decode_paged.restype = ctypes.c_int
         L.oracle_decode_paged.argtypes = [_D, _D, _D, _D, _D, _I, _I] + [ctypes.c_int] * 7
         L.oracle_decode.restype = ctypes.c_int
@@ -124,11 +130,12 @@ class Oracle:
     # -- Tylo.jl "Primitives" page, flex_attention! -----------------------------------
     def flex_fwd(self, Q, K, V, scale, causal=False, window=0, input_pos=0,
                  k_lengths=None, q_lengths=None, rows=None, Sq=None,
-                 softcap=0.0, alibi_slopes=None, doc_q=None, doc_kv=None):
-        """attn_fwd with SoftCapScore / AliBiScore and DocumentMask.
+                 softcap=0.0, alibi_slopes=None, doc_q=None, doc_kv=None, block_keep=None):
+        """attn_fwd with SoftCapScore / AliBiScore, DocumentMask and block sparsity.
 
         ``doc_q`` has one id per local query row (length Sq), ``doc_kv`` one per
-        key (length Sk); ``alibi_slopes`` one slope per query head.
+        key (length Sk); ``alibi_slopes`` one slope per query head; ``block_keep``
+        (B, Hq, ceil(Sq/64), ceil(Sk/64)) flags of the kept 64x64 blocks.
         """
         Q, K, V = _f64(Q), _f64(K), _f64(V)
         B, Hq, n, D = Q.shape
@@ -146,13 +153,18 @@ class Oracle:
         dq, dk = _i32(doc_q), _i32(doc_kv)
         if dq is not None:
             assert dq.shape == (Sq,) and dk is not None and dk.shape == (Sk,)
+        bk = None
+        if block_keep is not None:
+            bk = np.ascontiguousarray(np.asarray(block_keep, dtype=np.uint8))
+            assert bk.shape == (B, Hq, (Sq + 63) // 64, (Sk + 63) // 64)
         O = np.empty((B, Hq, n, D), dtype=np.float64)
         LSE = np.empty((B, Hq, n), dtype=np.float64)
         rc = self.lib.oracle_flex_fwd(_dptr(O), _dptr(LSE), _dptr(Q), _dptr(K), _dptr(V),
                                       B, Hq, Hkv, Sq, Sk, D, float(scale), int(causal),
                                       int(window), int(input_pos), _iptr(kl), _iptr(ql),
                                       _iptr(rows_a), n, float(softcap), _dptr(sl),
-                                      _iptr(dq), _iptr(dk))
+                                      _iptr(dq), _iptr(dk),
+                                      None if bk is None else bk.ctypes.data_as(ctypes.c_void_p))
         if rc != 0:
             raise ValueError("oracle_flex_fwd rejected its arguments")
         return O, LSE
@@ -172,6 +184,34 @@ class Oracle:
             raise ValueError("oracle_decode rejected its arguments")
         return O, LSE
 
+
+    # -- mlx-arsenal RBS page: block scores and the block mask --------------------------
+    def rbs_block_scores(self, Q, K):
+        """(base, rescue) log block scores, each (B, Hq, ceil(Sq/64), ceil(Sk/64))."""
+        Q, K = _f64(Q), _f64(K)
+        B, Hq, Sq, D = Q.shape
+        _, Hkv, Sk, _ = K.shape
+        nqb, nkb = (Sq + 63) // 64, (Sk + 63) // 64
+        base = np.empty((B, Hq, nqb, nkb), dtype=np.float64)
+        rescue = np.empty_like(base)
+        rc = self.lib.oracle_rbs_block_scores(_dptr(base), _dptr(rescue), _dptr(Q), _dptr(K),
+                                              B, Hq, Hkv, Sq, Sk, D)
+        if rc != 0:
+            raise ValueError("oracle_rbs_block_scores rejected its arguments")
+        return base, rescue
+
+    def rbs_block_mask(self, base, rescue, alpha_base=0.22, alpha_rescue=0.18, diagonal=1):
+        """uint8 keep flags of the RBS recipe (union of both branches and the band)."""
+        base, rescue = _f64(base), _f64(rescue)
+        *lead, nqb, nkb = base.shape
+        keep = np.empty(base.shape, dtype=np.uint8)
+        rows = int(np.prod(lead)) * nqb
+        rc = self.lib.oracle_rbs_block_mask(keep.ctypes.data_as(ctypes.c_void_p), _dptr(base),
+                                            _dptr(rescue), rows, nqb, nkb, float(alpha_base),
+                                            float(alpha_rescue), int(diagonal))
+        if rc != 0:
+            raise ValueError("oracle_rbs_block_mask rejected its arguments")
+        return keep
 
     # -- vllm-mlx paged KV cache + decode_attention! ------------------------------------
     def decode_paged(self, Q, K_cache, V_cache, block_tables, seq_lens):

@@ -36,6 +36,11 @@
  *     sequence b sits in block block_tables[b][j / block_size], slot
  *     j % block_size.  Decoding from it is decode_attention! over the tokens
  *     the block table gathers.
+ *   - mlx-arsenal "Radius-bounded block scores (RBS)" page: block centroids and
+ *     radii, the base and rescue log block scores per (query block, key block),
+ *     `relative_block_mask` and the recipe's union with a diagonal band; the
+ *     block-sparse attention that follows is `flex_attention!` with those
+ *     64x64 blocks masked.
  *   - Tylo.jl "Primitives" page, entry `decode_attention!`: one query vector
  *     per head and sequence against the first lengths[b] cached keys.  The
  *     split into n_splits slices and their combine change only the rounding,
@@ -56,6 +61,9 @@
  *     caller would fix; no such composition is built).  The ALiBi distance
  *     is (input_pos + i) - j, the absolute query position minus the key
  *     position, with the sign the page gives.
+ *   - RBS quantiles (median, 90th percentile) interpolate linearly between the
+ *     sorted radii (numpy's default); short last blocks average and score the
+ *     tokens they have.
  *   - document ids: doc_q[i] belongs to local query row i (absolute position
  *     input_pos + i), doc_kv[j] to key j; both are shared by every batch
  *     entry and head.
@@ -220,6 +228,8 @@ int oracle_attn_fwd(double *O, double *LSE, const double *Q, const double *K, co
  *                                                                (AliBiScore)
  *   visible_j = the causal / window / length rule of mask_row, and, if doc_q
  *               and doc_kv are given, doc_q[i] == doc_kv[j]       (DocumentMask)
+ *               and, if block_keep is given, the 64x64 block of (i, j) is kept
+ *               (block-sparse attention from a block mask per batch entry and head)
  *   then the softmax, O and LSE exactly as in oracle_attn_fwd.
  * Returns 0, or -1 on bad arguments.
  */
@@ -229,7 +239,8 @@ int oracle_flex_fwd(double *O, double *LSE, const double *Q, const double *K, co
                     const int *k_lengths, const int *q_lengths,
                     const int *rows, int n_rows,
                     double softcap, const double *alibi_slopes,
-                    const int *doc_q, const int *doc_kv) {
+                    const int *doc_q, const int *doc_kv,
+                    const unsigned char *block_keep) {
     if (B < 0 || Hq <= 0 || Hkv <= 0 || Sq < 0 || Sk < 0 || D <= 0) return -1;
     if (Hq % Hkv != 0) return -1;
     if (window > 0 && !causal) return -1;
@@ -271,6 +282,13 @@ int oracle_flex_fwd(double *O, double *LSE, const double *Q, const double *K, co
             if (doc_q != NULL)
                 for (long j = 0; j < Sk; ++j)
                     if (doc_q[i] != doc_kv[j]) mask[j] = -INFINITY;
+            if (block_keep != NULL) {
+                /* block-sparse attention: (B, Hq, ceil(Sq/64), ceil(Sk/64)) keep flags */
+                const long nqb = (Sq + 63) / 64, nkb = (Sk + 63) / 64;
+                const unsigned char *kr = block_keep + ((b * Hq + hq) * nqb + i / 64) * nkb;
+                for (long j = 0; j < Sk; ++j)
+                    if (!kr[j / 64]) mask[j] = -INFINITY;
+            }
             double mx = -INFINITY;
             for (long j = 0; j < Sk; ++j) {
                 double dot = 0.0;
@@ -448,4 +466,158 @@ int oracle_decode_paged(double *O, double *LSE, const double *Q, const double *K
         free(score);
     }
     return bad ? -1 : 0;
+}
+
+/*
+ * mlx-arsenal "Radius-bounded block scores (RBS)" page (sections "The idea" and
+ * "What mlx-arsenal ships"): block scores of block-sparse prefill.  For KV head
+ * h of batch b, key block kb (64 keys, the last one possibly shorter):
+ *   centroid c = mean of its keys, radius r = max over its keys of |k - c|_2;
+ *   r_low, r_high = median and 90th percentile of the head's block radii
+ *                   (linear interpolation between order statistics);
+ *   beta = clip((r - r_low) / (r_high - r_low), 0, 1), or, when r_high ==
+ *          r_low, 1 for r > r_low and 0 otherwise.
+ * For query head hq (KV head hq / (Hq/Hkv)) and query token t:
+ *   l_base   = <q_t, c> / sqrt(D)
+ *   l_rescue = (<q_t, c> + |q_t|_2 * r * beta) / sqrt(D)
+ * and the block scores are log sum_t exp(l) over the tokens t of query block qb.
+ *   Q (B, Hq, Sq, D); K (B, Hkv, Sk, D); base, rescue (B, Hq, nqb, nkb).
+ * Returns 0, or -1 on bad arguments.
+ */
+static int cmp_double(const void *a, const void *b) {
+    const double x = *(const double *)a, y = *(const double *)b;
+    return (x > y) - (x < y);
+}
+
+static double sorted_quantile(const double *v, int n, double q) {
+    const double pos = q * (n - 1);
+    const int lo = (int)floor(pos);
+    const int hi = lo + 1 < n ? lo + 1 : lo;
+    return v[lo] + (pos - lo) * (v[hi] - v[lo]);
+}
+
+int oracle_rbs_block_scores(double *base, double *rescue, const double *Q, const double *K,
+                            int B, int Hq, int Hkv, int Sq, int Sk, int D) {
+    if (B < 0 || Hq <= 0 || Hkv <= 0 || Sq < 0 || Sk <= 0 || D <= 0 || Hq % Hkv != 0) return -1;
+    const int BS = 64;
+    const int nqb = (Sq + BS - 1) / BS, nkb = (Sk + BS - 1) / BS;
+    const int group = Hq / Hkv;
+    const double inv_sqrt_d = 1.0 / sqrt((double)D);
+    double *cent = (double *)malloc(sizeof(double) * (size_t)B * Hkv * nkb * D);
+    double *rad = (double *)malloc(sizeof(double) * (size_t)B * Hkv * nkb);
+    double *beta = (double *)malloc(sizeof(double) * (size_t)B * Hkv * nkb);
+    if (!cent || !rad || !beta) {
+        free(cent); free(rad); free(beta);
+        return -1;
+    }
+    int bad = 0;
+#pragma omp parallel for schedule(dynamic, 1)
+    for (long bh = 0; bh < (long)B * Hkv; ++bh) {
+        const double *Kh = K + bh * (long)Sk * D;
+        for (int kb = 0; kb < nkb; ++kb) {
+            const int j0 = kb * BS, j1 = (j0 + BS < Sk) ? j0 + BS : Sk;
+            double *c = cent + (bh * nkb + kb) * (long)D;
+            for (int d = 0; d < D; ++d) {
+                double acc = 0.0;
+                for (int j = j0; j < j1; ++j) acc += Kh[(long)j * D + d];
+                c[d] = acc / (j1 - j0);
+            }
+            double rmax = 0.0;
+            for (int j = j0; j < j1; ++j) {
+                double ss = 0.0;
+                for (int d = 0; d < D; ++d) {
+                    const double e = Kh[(long)j * D + d] - c[d];
+                    ss += e * e;
+                }
+                if (sqrt(ss) > rmax) rmax = sqrt(ss);
+            }
+            rad[bh * nkb + kb] = rmax;
+        }
+        double *sorted = (double *)malloc(sizeof(double) * nkb);
+        if (!sorted) {
+#pragma omp atomic write
+            bad = 1;
+            continue;
+        }
+        memcpy(sorted, rad + bh * nkb, sizeof(double) * nkb);
+        qsort(sorted, nkb, sizeof(double), cmp_double);
+        const double r_low = sorted_quantile(sorted, nkb, 0.5);
+        const double r_high = sorted_quantile(sorted, nkb, 0.9);
+        free(sorted);
+        for (int kb = 0; kb < nkb; ++kb) {
+            const double r = rad[bh * nkb + kb];
+            double bt;
+            if (r_high > r_low) {
+                bt = (r - r_low) / (r_high - r_low);
+                bt = bt < 0.0 ? 0.0 : (bt > 1.0 ? 1.0 : bt);
+            } else {
+                bt = r > r_low ? 1.0 : 0.0;
+            }
+            beta[bh * nkb + kb] = bt;
+        }
+    }
+    if (!bad) {
+#pragma omp parallel for schedule(dynamic, 1)
+        for (long t = 0; t < (long)B * Hq * nqb; ++t) {
+            const long qb = t % nqb, hq = (t / nqb) % Hq, b = t / ((long)nqb * Hq);
+            const long bh = b * Hkv + hq / group;
+            const int i0 = (int)qb * BS, i1 = (i0 + BS < Sq) ? i0 + BS : Sq;
+            for (int kb = 0; kb < nkb; ++kb) {
+                const double *c = cent + (bh * nkb + kb) * (long)D;
+                const double rb = rad[bh * nkb + kb] * beta[bh * nkb + kb];
+                double mb = -INFINITY, mr = -INFINITY;
+                double lb[64], lr[64];
+                for (int i = i0; i < i1; ++i) {
+                    const double *q = Q + ((b * Hq + hq) * (long)Sq + i) * D;
+                    double dot = 0.0, qq = 0.0;
+                    for (int d = 0; d < D; ++d) {
+                        dot += q[d] * c[d];
+                        qq += q[d] * q[d];
+                    }
+                    lb[i - i0] = dot * inv_sqrt_d;
+                    lr[i - i0] = (dot + sqrt(qq) * rb) * inv_sqrt_d;
+                    if (lb[i - i0] > mb) mb = lb[i - i0];
+                    if (lr[i - i0] > mr) mr = lr[i - i0];
+                }
+                double sb = 0.0, sr = 0.0;
+                for (int i = 0; i < i1 - i0; ++i) {
+                    sb += exp(lb[i] - mb);
+                    sr += exp(lr[i] - mr);
+                }
+                base[t * nkb + kb] = mb + log(sb);
+                rescue[t * nkb + kb] = mr + log(sr);
+            }
+        }
+    }
+    free(cent); free(rad); free(beta);
+    return bad ? -1 : 0;
+}
+
+/*
+ * mlx-arsenal RBS page, `relative_block_mask(log_scores, alpha)` and the recipe
+ * `rbs_block_mask`: a block is kept when its summed exp over the query block
+ * is at least alpha times the row maximum, i.e. log_score >= max_row + ln alpha;
+ * the final mask is the union of the base branch (alpha_base), the rescue branch
+ * (alpha_rescue) and the band |qb - kb| < diagonal.  keep: 1 / 0 per block,
+ * rows = B * Hq * nqb rows of nkb blocks.
+ */
+int oracle_rbs_block_mask(unsigned char *keep, const double *base, const double *rescue,
+                          long rows, int nqb, int nkb, double alpha_base, double alpha_rescue,
+                          int diagonal) {
+    if (rows < 0 || nqb <= 0 || nkb <= 0 || !(alpha_base > 0.0) || !(alpha_rescue > 0.0)) return -1;
+    for (long r = 0; r < rows; ++r) {
+        const double *sb = base + r * nkb, *sr = rescue + r * nkb;
+        double mb = -INFINITY, mr = -INFINITY;
+        for (int k = 0; k < nkb; ++k) {
+            if (sb[k] > mb) mb = sb[k];
+            if (sr[k] > mr) mr = sr[k];
+        }
+        const long qb = r % nqb;
+        for (int k = 0; k < nkb; ++k) {
+            const int band = (qb - k < diagonal) && (k - qb < diagonal);
+            keep[r * nkb + k] = (sb[k] >= mb + log(alpha_base)) ||
+                                (sr[k] >= mr + log(alpha_rescue)) || band;
+        }
+    }
+    return 0;
 }

@@ -482,6 +482,89 @@ def pin_paged_reads_only_listed_slots(orc):
     assert np.all(np.isfinite(O1)) and np.array_equal(O1, O0) and np.array_equal(L1, L0)
 
 
+# --------------------------------------------------------------------------------------
+# mlx-arsenal "Radius-bounded block scores (RBS)" page: block scores and block mask;
+# block-sparse attention from a per-head block mask
+# --------------------------------------------------------------------------------------
+
+def pin_rbs_closed_form(orc):
+    """Key blocks built as c_b +/- delta_b e_1 (32 keys each way) have centroid c_b and
+    radius delta_b exactly; a query block of 64 identical tokens q scores
+    ln 64 + <q, c_b>/sqrt(D) (base) and ln 64 + (<q, c_b> + |q| delta_b beta_b)/sqrt(D)
+    (rescue), beta from the median and 90th percentile of the radii (numpy's
+    linear-interpolation quantile) clipped to [0, 1].  GQA: both query heads of
+    the KV head, with different q."""
+    rng = _rng(41)
+    D, nkb = 16, 10
+    deltas = np.arange(1, nkb + 1, dtype=np.float64) * 0.5
+    rng.shuffle(deltas)
+    cents = rng.standard_normal((nkb, D))
+    K = np.empty((1, 1, 64 * nkb, D))
+    for b in range(nkb):
+        sign = np.where(np.arange(64) % 2 == 0, 1.0, -1.0)
+        K[0, 0, 64 * b:64 * b + 64] = cents[b] + np.outer(sign, np.eye(D)[0]) * deltas[b]
+    qs = rng.standard_normal((2, D))
+    Q = np.repeat(qs[None, :, None, :], 64, axis=2)  # (1, 2, 64, D)
+    base, rescue = orc.rbs_block_scores(Q, K)
+    lo, hi = np.quantile(deltas, 0.5), np.quantile(deltas, 0.9)
+    beta = np.clip((deltas - lo) / (hi - lo), 0.0, 1.0)
+    for h in range(2):
+        q = qs[h]
+        want_b = math.log(64) + cents @ q / math.sqrt(D)
+        want_r = math.log(64) + (cents @ q + np.linalg.norm(q) * deltas * beta) / math.sqrt(D)
+        assert np.allclose(base[0, h, 0], want_b, rtol=0, atol=1e-10), h
+        assert np.allclose(rescue[0, h, 0], want_r, rtol=0, atol=1e-10), h
+
+
+def pin_rbs_degenerate_and_gqa(orc):
+    """Equal radii (the two quantiles coincide): no block is strictly wider, beta = 0,
+    rescue = base.  GQA: scores with 4 query heads on 2 KV heads equal those with the
+    KV heads repeated (4 on 4).  A short last block (Sq, Sk not multiples of 64)."""
+    rng = _rng(42)
+    D = 8
+    K = np.tile(rng.standard_normal((1, 1, 1, D)), (1, 1, 130, 1))  # every block radius 0
+    Q = rng.standard_normal((1, 2, 100, D))
+    base, rescue = orc.rbs_block_scores(Q, K)
+    assert np.array_equal(base, rescue)
+    Q = rng.standard_normal((2, 4, 150, D))
+    K = rng.standard_normal((2, 2, 200, D))
+    b1, r1 = orc.rbs_block_scores(Q, K)
+    b2, r2 = orc.rbs_block_scores(Q, np.repeat(K, 2, axis=1))
+    assert np.max(np.abs(b1 - b2)) < 1e-12 and np.max(np.abs(r1 - r2)) < 1e-12
+
+
+def pin_rbs_relative_mask_golden(orc):
+    """Hand-derived union of the two relative masks and the band
+    (golden/rbs_relative_mask.json)."""
+    with open(os.path.join(GOLDEN, "rbs_relative_mask.json")) as f:
+        g = json.load(f)
+    base = np.log(np.array(g["base_ratio"], dtype=np.float64))[None, None]
+    rescue = np.log(np.array(g["rescue_ratio"], dtype=np.float64))[None, None]
+    keep = orc.rbs_block_mask(base, rescue, g["alpha_base"], g["alpha_rescue"], g["diagonal"])
+    assert np.array_equal(keep[0, 0], np.array(g["keep"], dtype=np.uint8)), keep
+
+
+def pin_block_sparse_attention(orc):
+    """Keeping every block is attention!; keeping only the 64x64 diagonal blocks is
+    attention! on each 64-token block alone (per head: head 1 keeps everything)."""
+    rng = _rng(43)
+    S, D = 150, 8
+    Q, K, V = rng.standard_normal((1, 2, S, D)), rng.standard_normal((1, 2, S, D)), \
+        rng.standard_normal((1, 2, S, D))
+    nb = (S + 63) // 64
+    keep = np.ones((1, 2, nb, nb), dtype=np.uint8)
+    O0, L0 = orc.attn_fwd(Q, K, V, 0.3)
+    O1, L1 = orc.flex_fwd(Q, K, V, 0.3, block_keep=keep)
+    assert np.max(np.abs(O1 - O0)) < 1e-12 and np.max(np.abs(L1 - L0)) < 1e-12
+    keep[0, 0] = np.eye(nb, dtype=np.uint8)
+    O2, L2 = orc.flex_fwd(Q, K, V, 0.3, block_keep=keep)
+    assert np.max(np.abs(O2[0, 1] - O0[0, 1])) < 1e-12
+    for a in range(0, S, 64):
+        sl = slice(a, min(a + 64, S))
+        Ob, Lb = orc.attn_fwd(Q[:, :1, sl], K[:, :1, sl], V[:, :1, sl], 0.3)
+        assert np.max(np.abs(O2[:, :1, sl] - Ob)) < 1e-12 and np.max(np.abs(L2[:, :1, sl] - Lb)) < 1e-12
+
+
 PINS = [
     pin_causal_mask_shape_and_rows,
     pin_sliding_window_rows,
@@ -503,4 +586,8 @@ PINS = [
     pin_flex_document_blocks,
     pin_paged_equals_contiguous,
     pin_paged_reads_only_listed_slots,
+    pin_rbs_closed_form,
+    pin_rbs_degenerate_and_gqa,
+    pin_rbs_relative_mask_golden,
+    pin_block_sparse_attention,
 ]

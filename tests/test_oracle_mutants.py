@@ -63,6 +63,20 @@ MUTANTS = {
     "paged_scale": ("const double qk_scale = 1.0 / sqrt((double)D);", "const double qk_scale = 1.0 / (double)D;"),
     "paged_lse_missing_max": ("if (LSE) LSE[b * Hq + hq] = mx + log(den);",
                               "if (LSE) LSE[b * Hq + hq] = log(den);"),
+    "rbs_centroid_sum": ("c[d] = acc / (j1 - j0);", "c[d] = acc / BS;"),
+    "rbs_radius_squared": ("if (sqrt(ss) > rmax) rmax = sqrt(ss);", "if (ss > rmax) rmax = ss;"),
+    "rbs_quantile_low": ("sorted_quantile(sorted, nkb, 0.5);", "sorted_quantile(sorted, nkb, 0.4);"),
+    "rbs_beta_unclipped": ("bt = bt < 0.0 ? 0.0 : (bt > 1.0 ? 1.0 : bt);", "bt = bt;"),
+    "rbs_degenerate_beta": ("bt = r > r_low ? 1.0 : 0.0;", "bt = 1.0;"),
+    "rbs_rescue_no_norm": ("lr[i - i0] = (dot + sqrt(qq) * rb) * inv_sqrt_d;",
+                           "lr[i - i0] = (dot + rb) * inv_sqrt_d;"),
+    "rbs_scale": ("const double inv_sqrt_d = 1.0 / sqrt((double)D);", "const double inv_sqrt_d = 1.0 / (double)D;"),
+    "rbs_lse_max_only": ("base[t * nkb + kb] = mb + log(sb);", "base[t * nkb + kb] = mb;"),
+    "rbs_gqa_modulo": ("const long bh = b * Hkv + hq / group;", "const long bh = b * Hkv + hq % Hkv;"),
+    "mask_alpha_inverted": ("(sb[k] >= mb + log(alpha_base))", "(sb[k] >= mb - log(alpha_base))"),
+    "mask_band_wide": ("(qb - k < diagonal) && (k - qb < diagonal)", "(qb - k <= diagonal) && (k - qb <= diagonal)"),
+    "mask_no_rescue": ("(sr[k] >= mr + log(alpha_rescue)) || band", "band"),
+    "block_keep_ignored": ("if (!kr[j / 64]) mask[j] = -INFINITY;", "if (0) mask[j] = -INFINITY;"),
 }
 
 
