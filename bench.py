@@ -405,6 +405,58 @@ def time_flex(dev, steps, warmup, peak):
     return out
 
 
+def time_block_sparse(dev, steps, warmup, peak):
+    """Block-sparse prefill row on the block-structured image workload: RBS block scores + mask
+    (attn_rbs_block_mask), then attention over the kept 64x64 blocks (attn_fwd_flex,
+    per-head masks); CUDA events per launch.  TFLOP/s counts the kept pairs; the
+    dense attention of the same inputs is timed beside it."""
+    from gqa_attention_flash_b200 import binding
+    w = W.BLOCK_SPARSE
+    x = W.make_prefill(w)
+    Q, K, V = x.Q.to(dev), x.K.to(dev), x.V.to(dev)
+    O = torch.empty_like(Q)
+    L = torch.empty(Q.shape[:3], dtype=torch.float32, device=dev)
+    holder = {}
+
+    def est():
+        holder["mask"] = binding.rbs_block_mask(Q, K)
+
+    def sparse():
+        binding.attn_fwd_flex(O, Q, K, V, L, w.scale, False, block_mask=holder["mask"])
+
+    def dense():
+        binding.attn_fwd(O, Q, K, V, L, w.scale, False)
+
+    def timed(fn):
+        for _ in range(warmup):
+            fn()
+        torch.cuda.synchronize()
+        ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+              for _ in range(steps)]
+        for e0, e1 in ev:
+            e0.record()
+            fn()
+            e1.record()
+        torch.cuda.synchronize()
+        return sum(a.elapsed_time(b) for a, b in ev) / steps
+    t_est = timed(est)
+    t_sparse = timed(sparse)
+    t_dense = timed(dense)
+    st = binding.last_device_status()
+    if st != 0:
+        raise RuntimeError(f"block-sparse device status: {binding.status_string(st)}")
+    kept = int((holder["mask"] == 2).sum())
+    total = holder["mask"].numel()
+    kept_flops = 4 * w.D * kept * 64 * 64  # S = 4096: every block is a full 64 x 64 block
+    tf = kept_flops / (t_sparse * 1e-3) / 1e12
+    return {"workload": w.name + ", RBS alpha 0.22 / 0.18, band 1", "value": tf,
+            "unit": "TFLOP/s (kept blocks)", "density": kept / total,
+            "estimator_ms": t_est, "sparse_attention_ms": t_sparse, "dense_attention_ms": t_dense,
+            "speedup_vs_dense": t_dense / (t_est + t_sparse), "launches": steps,
+            "roofline": {"bound": "tensor", "achieved": tf, "peak": peak, "unit": "TFLOP/s",
+                         "frac": tf / peak, "kernel": "attn_fwd_kernel<128, flex, block list>"}}
+
+
 def time_paged(step, steps, warmup, peak):
     """Paged-KV decode row: the step's decode sequences scattered into a shuffled
     pool of 16-token blocks (block tables), device-resident; CUDA events around
@@ -567,8 +619,11 @@ def main(argv=None):
     if args.only == "flex":
         peaks, _ = load_peaks()
         res = time_flex(dev, args.steps, args.warmup, peaks["bf16_tflops"])
+        bs = time_block_sparse(dev, args.steps, args.warmup, peaks["bf16_tflops"])
         print(json.dumps({"profiling_run": True,
-                          "flex_ms": {k: v["ms_per_launch"] for k, v in res.items()}}), flush=True)
+                          "flex_ms": {k: v["ms_per_launch"] for k, v in res.items()},
+                          "block_sparse_ms": [bs["estimator_ms"], bs["sparse_attention_ms"]]}),
+              flush=True)
         return 0
     step = Step(dev, args.only, args.decode_batch)
     profiling = args.only is not None or args.decode_batch is not None
@@ -637,6 +692,9 @@ def main(argv=None):
         line["cpu_baseline"] = cpu_baseline(step.host_prefill, step.dQ_host, step.lengths_host)
     if not args.no_flex:
         line["flex"] = time_flex(dev, min(K, 50), args.warmup, peaks["bf16_tflops"])
+    if not args.no_flex:
+        line["block_sparse"] = time_block_sparse(dev, min(K, 50), args.warmup,
+                                                 peaks["bf16_tflops"])
     if not args.no_paged and step.do_decode:
         line["paged_decode"] = time_paged(step, min(K, 100), args.warmup, peaks["hbm_gbs"])
     print(json.dumps(line), flush=True)

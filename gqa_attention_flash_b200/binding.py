@@ -36,7 +36,9 @@ lib.attn_fwd_varlen.restype = _i
 lib.attn_fwd_varlen.argtypes = [_p, _p, _p, _p, _p] + [_i] * 6 + [_f, _i, _i, _i, _p, _p, _p]
 lib.attn_fwd_flex.restype = _i
 lib.attn_fwd_flex.argtypes = [_p, _p, _p, _p, _p] + [_i] * 6 + [_f, _i, _i, _i, _p, _p, _f, _p, _p,
-                                                                _p, _p, _p]
+                                                                _p, _p, _i, _p]
+lib.attn_rbs_block_mask.restype = _i
+lib.attn_rbs_block_mask.argtypes = [_p, _p, _p, _p, _p] + [_i] * 6 + [_f, _f, _i, _p]
 _KEEP = ctypes.CFUNCTYPE(_i, _i, _i, _p)
 lib.attn_block_mask_build.restype = _i
 lib.attn_block_mask_build.argtypes = [_p, _i, _i, _i, _KEEP, _p]
@@ -105,15 +107,34 @@ def attn_fwd_flex(O, Q, K, V, LSE, scale, causal=False, window=0, input_pos=0, k
                   block_mask=None, stream=None):
     """flex_attention! forward: attn_fwd plus SoftCapScore (softcap > 0) or
     AliBiScore (alibi_slopes, fp32 (Hq,)), DocumentMask (doc_q int32 (Sq,), doc_kv
-    int32 (Sk,)) and a BlockMask (uint8 (ceil(Sq/64), ceil(Sk/64))), all on the
-    device."""
+    int32 (Sk,)) and a BlockMask (uint8 (ceil(Sq/64), ceil(Sk/64)), or one per
+    (batch, query head) as a 4-D (B, Hq, ., .) tensor), all on the device."""
     B, Hq, Sq, D = Q.shape
     _, Hkv, Sk, _ = K.shape
     rc = lib.attn_fwd_flex(_ptr(O), _ptr(Q), _ptr(K), _ptr(V), _ptr(LSE), B, Hq, Hkv, Sq, Sk, D,
                            float(scale), int(causal), int(window), int(input_pos),
                            _ptr(k_lengths), _ptr(q_lengths), float(softcap), _ptr(alibi_slopes),
-                           _ptr(doc_q), _ptr(doc_kv), _ptr(block_mask), _stream(stream))
+                           _ptr(doc_q), _ptr(doc_kv), _ptr(block_mask),
+                           1 if block_mask is not None and block_mask.dim() == 4 else 0,
+                           _stream(stream))
     _check(rc, "attn_fwd_flex")
+
+
+def rbs_block_mask(Q, K, alpha_base=0.22, alpha_rescue=0.18, diagonal=1, want_scores=False,
+                   stream=None):
+    """Block-sparse prefill mask from the RBS block scores: uint8 (B, Hq, nqb, nkb)
+    device tensor (2 = keep, 0 = skip), plus the (base, rescue) scores if asked."""
+    B, Hq, Sq, D = Q.shape
+    _, Hkv, Sk, _ = K.shape
+    shape = (B, Hq, (Sq + 63) // 64, (Sk + 63) // 64)
+    mask = torch.empty(shape, dtype=torch.uint8, device=Q.device)
+    base = torch.empty(shape, dtype=torch.float32, device=Q.device) if want_scores else None
+    resc = torch.empty(shape, dtype=torch.float32, device=Q.device) if want_scores else None
+    rc = lib.attn_rbs_block_mask(_ptr(mask), _ptr(base), _ptr(resc), _ptr(Q), _ptr(K), B, Hq,
+                                 Hkv, Sq, Sk, D, float(alpha_base), float(alpha_rescue),
+                                 int(diagonal), _stream(stream))
+    _check(rc, "attn_rbs_block_mask")
+    return (mask, base, resc) if want_scores else mask
 
 
 def block_mask_shape(Sq: int, Sk: int):

@@ -194,13 +194,14 @@ attn_status_t attn_fwd_flex(void *O, const void *Q, const void *K, const void *V
                             const int32_t *k_lengths, const int32_t *q_lengths,
                             float softcap, const float *alibi_slopes,
                             const int32_t *doc_q, const int32_t *doc_kv,
-                            const uint8_t *block_mask, void *stream) {
+                            const uint8_t *block_mask, int block_mask_per_head, void *stream) {
     attn_status_t st =
         validate_fwd(O, Q, K, V, LSE, B, Hq, Hkv, Sq, Sk, D, scale, causal, window, input_pos);
     if (st != ATTN_OK) return st;
     if (!(softcap >= 0.f) || !std::isfinite(softcap)) return ATTN_ERR_INVALID;
     if (softcap > 0.f && alibi_slopes) return ATTN_ERR_INVALID;
     if ((doc_q == nullptr) != (doc_kv == nullptr)) return ATTN_ERR_INVALID;
+    if (block_mask_per_head != 0 && block_mask_per_head != 1) return ATTN_ERR_INVALID;
     if ((reinterpret_cast<uintptr_t>(alibi_slopes) | reinterpret_cast<uintptr_t>(doc_q) |
          reinterpret_cast<uintptr_t>(doc_kv)) & 3u)
         return ATTN_ERR_INVALID;
@@ -230,6 +231,7 @@ attn_status_t attn_fwd_flex(void *O, const void *Q, const void *K, const void *V
     a.doc_q = doc_q;
     a.doc_kv = doc_kv;
     a.block_mask = block_mask;
+    a.block_mask_per_head = block_mask_per_head;
     if (Sk == 0) {
         a.K = Q;  // stand-in tensor map; no key is visible
         a.V = Q;
@@ -272,6 +274,50 @@ attn_status_t attn_decode(void *O, const void *Q, const void *K, const void *V,
     a.D = D;
     a.workspace = static_cast<float *>(ws);
     attn_status_t st = launch_decode(a, s);
+    if (cudaFreeAsync(ws, s) != cudaSuccess && st == ATTN_OK) st = ATTN_ERR_CUDA;
+    return st;
+}
+
+attn_status_t attn_rbs_block_mask(uint8_t *block_mask, float *base_scores, float *rescue_scores,
+                                  const void *Q, const void *K, int B, int Hq, int Hkv, int Sq,
+                                  int Sk, int D, float alpha_base, float alpha_rescue,
+                                  int diagonal, void *stream) {
+    if (B < 0 || Hq < 1 || Hkv < 1 || Sq < 0 || Sk < 0 || diagonal < 0) return ATTN_ERR_INVALID;
+    if (Hq % Hkv != 0) return ATTN_ERR_INVALID;
+    if (!(alpha_base > 0.f) || !(alpha_rescue > 0.f) || !std::isfinite(alpha_base) ||
+        !std::isfinite(alpha_rescue))
+        return ATTN_ERR_INVALID;
+    if (D != 64 && D != 128) return ATTN_ERR_UNSUPPORTED;
+    if ((long long)Sk > 131072) return ATTN_ERR_UNSUPPORTED;
+    if ((long long)B * Hq * Sq == 0 || Sk == 0) return ATTN_OK;
+    if (!block_mask || !Q || !K) return ATTN_ERR_NULL;
+    if (!aligned16(Q) || !aligned16(K) ||
+        ((reinterpret_cast<uintptr_t>(base_scores) | reinterpret_cast<uintptr_t>(rescue_scores)) & 3u))
+        return ATTN_ERR_INVALID;
+    const long long nkb = (Sk + 63) / 64;
+    const size_t ws_floats = (size_t)B * Hkv * nkb * (D + 2);
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    void *ws = nullptr;
+    if (cudaMallocAsync(&ws, ws_floats * sizeof(float), s) != cudaSuccess) return ATTN_ERR_CUDA;
+    RbsArgs a;
+    a.Q = Q;
+    a.K = K;
+    a.B = B;
+    a.Hq = Hq;
+    a.Hkv = Hkv;
+    a.Sq = Sq;
+    a.Sk = Sk;
+    a.D = D;
+    a.alpha_base = alpha_base;
+    a.alpha_rescue = alpha_rescue;
+    a.diagonal = diagonal;
+    a.mask = block_mask;
+    a.base_scores = base_scores;
+    a.rescue_scores = rescue_scores;
+    a.cent = static_cast<float *>(ws);
+    a.rad = a.cent + (size_t)B * Hkv * nkb * D;
+    a.beta = a.rad + (size_t)B * Hkv * nkb;
+    attn_status_t st = launch_rbs(a, s);
     if (cudaFreeAsync(ws, s) != cudaSuccess && st == ATTN_OK) st = ATTN_ERR_CUDA;
     return st;
 }

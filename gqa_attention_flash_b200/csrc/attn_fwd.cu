@@ -98,6 +98,7 @@ struct FwdParams {
     const int32_t *doc_kv;   // ... per key, or null
     const uint8_t *bmask;    // BlockMask states of 64x64 blocks (n_qb, n_kb), or null
     int n_qb, n_kb;
+    int bmask_per_head;      // bmask holds one (n_qb, n_kb) matrix per (batch, query head)
 };
 
 // flex_attention!: 2-bit states of the four 64x64 blocks of the 128x128 tile
@@ -105,7 +106,8 @@ struct FwdParams {
 // the document mask), 2 = every pair the block mask covers is visible.  State of
 // block (query half qs, key half ks) sits at bits 2 * (2 qs + ks).  Blocks past
 // the ends of the BlockMask are 0.
-__device__ __forceinline__ uint32_t flex_states(const FwdParams &p, int qt, int u) {
+__device__ __forceinline__ uint32_t flex_states(const FwdParams &p, const uint8_t *bm, int qt,
+                                                int u) {
     uint32_t st = 0;
 #pragma unroll
     for (int qs = 0; qs < 2; ++qs)
@@ -114,8 +116,8 @@ __device__ __forceinline__ uint32_t flex_states(const FwdParams &p, int qt, int 
             const int qb = 2 * qt + qs, kb = 2 * u + ks;
             uint32_t v = 0;
             if (qb < p.n_qb && kb < p.n_kb) {
-                if (p.bmask) {
-                    const uint32_t m = p.bmask[(size_t)qb * p.n_kb + kb];
+                if (bm) {
+                    const uint32_t m = bm[(size_t)qb * p.n_kb + kb];
                     v = m == 0 ? 0u : (m == 2 ? 2u : 1u);
                 } else {
                     v = p.doc_q ? 1u : 2u;
@@ -246,13 +248,15 @@ __global__ void __launch_bounds__(kThreads, 1)
         // The KV tiles this CTA visits: inside a query tile's analytic range and
         // holding a visible block (BlockMask of flex_attention!), in order.
         if (warp == kWarpTma) {
+            const uint8_t *bm = p.bmask;
+            if (bm && p.bmask_per_head) bm += (size_t)(b * p.Hq + hq) * p.n_qb * p.n_kb;
             int count = 0;
             for (int base = u_lo; n_u > 0 && base < u_hi; base += 32) {
                 const int u = base + lane;
                 uint32_t e = 0;
                 if (u < u_hi) {
-                    const uint32_t s0 = USES(0, u) ? flex_states(p, pair * kTiles, u) : 0u;
-                    const uint32_t s1 = USES(1, u) ? flex_states(p, pair * kTiles + 1, u) : 0u;
+                    const uint32_t s0 = USES(0, u) ? flex_states(p, bm, pair * kTiles, u) : 0u;
+                    const uint32_t s1 = USES(1, u) ? flex_states(p, bm, pair * kTiles + 1, u) : 0u;
                     if (s0 | s1) e = static_cast<uint32_t>(u) | (s0 << 16) | (s1 << 24);
                 }
                 const uint32_t vote = __ballot_sync(0xffffffffu, e != 0);
@@ -739,6 +743,7 @@ attn_status_t launch_fwd_d(const FwdArgs &a, cudaStream_t stream) {
     p.doc_q = a.doc_q;
     p.doc_kv = a.doc_kv;
     p.bmask = a.block_mask;
+    p.bmask_per_head = a.block_mask_per_head;
     p.n_qb = (a.Sq + 63) / 64;
     p.n_kb = (a.Sk + 63) / 64;
     if (!p.status) return ATTN_ERR_CUDA;

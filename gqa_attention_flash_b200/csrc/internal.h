@@ -34,6 +34,7 @@ struct FwdArgs {
     const float *alibi_slopes = nullptr;
     const int32_t *doc_q = nullptr, *doc_kv = nullptr;
     const uint8_t *block_mask = nullptr;
+    int block_mask_per_head = 0;  // block_mask is (B, Hq, nqb, nkb) instead of (nqb, nkb)
 };
 
 // Longest KV sequence the flex kernel takes, in 128-key tiles (its per-CTA list
@@ -52,6 +53,19 @@ struct DecodeArgs {
     const int32_t *block_tables = nullptr;
     int num_blocks = 0, block_size = 0, max_blocks = 0;
 };
+
+// Block scores + block mask of block-sparse prefill (RBS page of mlx-arsenal).
+struct RbsArgs {
+    const void *Q, *K;
+    int B, Hq, Hkv, Sq, Sk, D;
+    float alpha_base, alpha_rescue;
+    int diagonal;
+    uint8_t *mask;                     // (B, Hq, nqb, nkb) BlockMask states 2 / 0
+    float *base_scores, *rescue_scores;  // (B, Hq, nqb, nkb) or nullptr
+    float *cent, *rad, *beta;          // workspace: (B, Hkv, nkb, D), (B, Hkv, nkb) x 2
+};
+
+attn_status_t launch_rbs(const RbsArgs &a, cudaStream_t stream);
 
 // Device address of the status word on the current device (looked up once per
 // device), or nullptr if the lookup failed.

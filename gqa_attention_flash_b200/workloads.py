@@ -52,6 +52,7 @@ class PrefillWorkload:
     ragged: tuple | None = None           # (lo, hi) inclusive range for k_len = q_len
     block_offset_std: float = 0.0         # image workload: per-64-token-block K offset
     block: int = 64
+    q_block_offset_std: float = 0.0       # per-64-token-block Q offset (block-structured)
 
     def flops(self, k_lengths=None, q_lengths=None) -> int:
         """Algorithmic FLOPs: 4 * D * (number of visible (query, key) pairs)."""
@@ -84,6 +85,11 @@ IMAGE = PrefillWorkload("image-image non-causal B1 H32 S4096 D128 (64x64 tokens)
                         block_offset_std=0.5)
 DECODE = DecodeWorkload("split-KV decode B64 Hq32 Hkv8 D128 cap32768 n_splits8", 64, 32, 8,
                         32768, 128, 8, 1024, 32768, seed=4)
+
+BLOCK_SPARSE = PrefillWorkload("block-structured image attention B1 H32 S4096 D128: Q and K "
+                               "offsets per 64-token block ~ N(0, 1.5^2)", 1, 32, 32, 4096, 4096,
+                               128, 1.0 / math.sqrt(128.0), False, seed=8, block_offset_std=1.5,
+                               q_block_offset_std=1.5)
 
 PREFILL_WORKLOADS = {"tiny": TINY, "llm": LLM, "window": WINDOW, "image": IMAGE}
 
@@ -177,6 +183,10 @@ def make_prefill(w: PrefillWorkload) -> PrefillInputs:
         nblk = (w.Sk + w.block - 1) // w.block
         c = torch.randn(w.Hkv, nblk, w.D, generator=g, dtype=torch.float32) * w.block_offset_std
         K = K + c.repeat_interleave(w.block, dim=1)[:, :w.Sk].unsqueeze(0)
+    if w.q_block_offset_std > 0:
+        nqb = (w.Sq + w.block - 1) // w.block
+        cq = torch.randn(w.Hq, nqb, w.D, generator=g, dtype=torch.float32) * w.q_block_offset_std
+        Q = Q + cq.repeat_interleave(w.block, dim=1)[:, :w.Sq].unsqueeze(0)
     k_len = q_len = None
     if w.ragged is not None:
         lo, hi = w.ragged

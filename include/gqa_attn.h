@@ -117,6 +117,10 @@ attn_status_t attn_fwd_varlen(void *O, const void *Q, const void *K, const void 
  *                 ids not checked), anything else = check each pair.  Build it
  *                 with attn_block_mask_document or attn_block_mask_build (the
  *                 page's build_block_mask); it must agree with the other masks.
+ *   block_mask_per_head  0: one block_mask for every batch entry and head;
+ *                 1: block_mask is (B, Hq, ceil(Sq/64), ceil(Sk/64)), one matrix
+ *                 per (batch, query head) -- block-sparse prefill with the
+ *                 masks of attn_rbs_block_mask.
  * Limits: Sk <= 131072.  Errors as attn_fwd, plus ATTN_ERR_INVALID for a
  * negative or non-finite softcap, softcap together with ALiBi, or only one of
  * doc_q / doc_kv, and ATTN_ERR_UNSUPPORTED for a longer Sk.
@@ -127,7 +131,34 @@ attn_status_t attn_fwd_flex(void *O, const void *Q, const void *K, const void *V
                             const int32_t *k_lengths, const int32_t *q_lengths,
                             float softcap, const float *alibi_slopes,
                             const int32_t *doc_q, const int32_t *doc_kv,
-                            const uint8_t *block_mask, void *stream);
+                            const uint8_t *block_mask, int block_mask_per_head, void *stream);
+
+/*
+ * attn_rbs_block_mask -- block scores and block mask of block-sparse prefill
+ * (mlx-arsenal "Radius-bounded block scores (RBS)" page: the block estimator of
+ * "The idea", radius_bounded_block_scores and relative_block_mask of "What
+ * mlx-arsenal ships", and the union of the recipe), 64-token blocks.
+ *
+ *   block_mask  [out] uint8 (B, Hq, ceil(Sq/64), ceil(Sk/64)) device array:
+ *               2 = keep the block, 0 = skip it; pass it to attn_fwd_flex with
+ *               block_mask_per_head = 1.
+ *   base_scores, rescue_scores [out] float32, same shape, or NULL: the log
+ *               block scores log sum_t exp(l_t) over the query block's tokens,
+ *               l_base = <q, c> / sqrt(D), l_rescue = (<q, c> + |q| r beta) /
+ *               sqrt(D), c / r the key block's centroid / radius, beta =
+ *               clip((r - r_low) / (r_high - r_low), 0, 1) with r_low / r_high
+ *               the median / 90th percentile of the KV head's block radii.
+ *   Q (B, Hq, Sq, D), K (B, Hkv, Sk, D) bf16 device arrays (GQA: query head h
+ *               scores the blocks of KV head h / (Hq / Hkv)).
+ *   A block is kept when base >= row max + ln alpha_base, or rescue >= row max
+ *   + ln alpha_rescue, or |qb - kb| < diagonal (the page uses 0.22, 0.18, 1).
+ * Limits: Sk <= 131072, D in {64, 128}.  Allocates a stream-ordered workspace
+ * of B * Hkv * ceil(Sk/64) * (D + 2) floats.
+ */
+attn_status_t attn_rbs_block_mask(uint8_t *block_mask, float *base_scores, float *rescue_scores,
+                                  const void *Q, const void *K, int B, int Hq, int Hkv, int Sq,
+                                  int Sk, int D, float alpha_base, float alpha_rescue,
+                                  int diagonal, void *stream);
 
 /*
  * attn_block_mask_build -- the page's build_block_mask (Tylo.jl "Primitives"

@@ -107,7 +107,7 @@ def flex(binding, **kw):
                                      a["Hkv"], a["Sq"], a["Sk"], a["D"], a["scale"], a["causal"],
                                      a["window"], a["input_pos"], a["k_lengths"], a["q_lengths"],
                                      a["softcap"], a["alibi"], a["doc_q"], a["doc_kv"],
-                                     a["block_mask"], None)
+                                     a["block_mask"], a.get("per_head", 0), None)
 
 
 def test_flex_host_validation(binding):
@@ -121,6 +121,7 @@ def test_flex_host_validation(binding):
     assert flex(binding, doc_kv=P) == 2
     assert flex(binding, alibi=ctypes.c_void_p(18)) == 2  # misaligned slopes
     assert flex(binding, Sk=128 * 1024 + 1) == 3          # longer than the flex kernel takes
+    assert flex(binding, per_head=2) == 2
     assert flex(binding, B=0) == 0
     assert flex(binding, Sq=0, softcap=3.0) == 0
 
@@ -197,3 +198,24 @@ def test_paged_layout_helper():
     for b, ln in enumerate(lengths):
         nb = (ln + 15) // 16
         assert bool((tables[b, :nb] >= 0).all()) and bool((tables[b, nb:] == -1).all())
+
+
+def test_rbs_host_validation(binding):
+    L = binding.lib
+
+    def rbs(**kw):
+        a = dict(mask=P, base=None, resc=None, Q=P, K=P, B=1, Hq=4, Hkv=2, Sq=128, Sk=128, D=128,
+                 ab=0.22, ar=0.18, diag=1)
+        a.update(kw)
+        return L.attn_rbs_block_mask(a["mask"], a["base"], a["resc"], a["Q"], a["K"], a["B"],
+                                     a["Hq"], a["Hkv"], a["Sq"], a["Sk"], a["D"], a["ab"], a["ar"],
+                                     a["diag"], None)
+    assert rbs(Hq=3) == 2
+    assert rbs(ab=0.0) == 2
+    assert rbs(ar=float("nan")) == 2
+    assert rbs(diag=-1) == 2
+    assert rbs(D=96) == 3
+    assert rbs(Sk=131073) == 3
+    assert rbs(mask=None) == 1
+    assert rbs(Q=ctypes.c_void_p(20)) == 2
+    assert rbs(B=0) == 0
