@@ -80,6 +80,9 @@ class Oracle:
                                             ctypes.c_int]
         L.oracle_decode_paged.restype = ctypes.c_int
         L.oracle_decode_paged.argtypes = [_D, _D, _D, _D, _D, _I, _I] + [ctypes.c_int] * 7
+        L.oracle_attn_bwd.restype = ctypes.c_int
+        L.oracle_attn_bwd.argtypes = [_D] * 7 + [ctypes.c_int] * 6 + [
+            ctypes.c_double, ctypes.c_int, ctypes.c_int, ctypes.c_int, _I, _I]
         L.oracle_decode.restype = ctypes.c_int
         L.oracle_decode.argtypes = [_D, _D, _D, _D, _D] + [ctypes.c_int] * 5 + [_I]
 
@@ -184,6 +187,24 @@ class Oracle:
             raise ValueError("oracle_decode rejected its arguments")
         return O, LSE
 
+
+    # -- Tylo.jl "Primitives" page, ∇attention! ---------------------------------------
+    def attn_bwd(self, Q, K, V, dO, scale, causal=False, window=0, input_pos=0,
+                 k_lengths=None, q_lengths=None):
+        """(dQ, dK, dV) float64 for the output gradient dO (shapes of Q, K, V, O)."""
+        Q, K, V, dO = _f64(Q), _f64(K), _f64(V), _f64(dO)
+        B, Hq, Sq, D = Q.shape
+        _, Hkv, Sk, _ = K.shape
+        assert dO.shape == Q.shape and V.shape == K.shape
+        kl, ql = _i32(k_lengths), _i32(q_lengths)
+        dQ, dK, dV = np.empty_like(Q), np.empty_like(K), np.empty_like(V)
+        rc = self.lib.oracle_attn_bwd(_dptr(dQ), _dptr(dK), _dptr(dV), _dptr(Q), _dptr(K),
+                                      _dptr(V), _dptr(dO), B, Hq, Hkv, Sq, Sk, D, float(scale),
+                                      int(causal), int(window), int(input_pos), _iptr(kl),
+                                      _iptr(ql))
+        if rc != 0:
+            raise ValueError("oracle_attn_bwd rejected its arguments")
+        return dQ, dK, dV
 
     # -- mlx-arsenal RBS page: block scores and the block mask --------------------------
     def rbs_block_scores(self, Q, K):

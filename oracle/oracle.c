@@ -41,6 +41,12 @@
  *     `relative_block_mask` and the recipe's union with a diagonal band; the
  *     block-sparse attention that follows is `flex_attention!` with those
  *     64x64 blocks masked.
+ *   - Tylo.jl "Primitives" page, entry `∇attention!`: the input gradients of
+ *     attention! from the output gradient: with P the softmax probabilities,
+ *     dV = P^T dO, dP = dO V^T, dS = P * (dP - rowsum(dP * P)), dQ = scale dS K,
+ *     dK = scale dS^T Q (GQA: a KV head collects the gradients of all the query
+ *     heads it serves).  The oracle recomputes P from its definition; the GPU
+ *     uses the saved LSE, which gives the same P up to rounding.
  *   - Tylo.jl "Primitives" page, entry `decode_attention!`: one query vector
  *     per head and sequence against the first lengths[b] cached keys.  The
  *     split into n_splits slices and their combine change only the rounding,
@@ -620,4 +626,93 @@ int oracle_rbs_block_mask(unsigned char *keep, const double *base, const double 
         }
     }
     return 0;
+}
+
+/*
+ * Tylo.jl "Primitives" page, `∇attention!`: gradients of the attention! rows
+ * defined above (same masks and lengths) for the output gradient dO.
+ *   per (b, hq, row i):  P_i = softmax(S_i + mask_i)      (explicit row)
+ *                        dP_ij = <dO_i, V_j>
+ *                        delta_i = sum_j P_ij dP_ij
+ *                        dS_ij = P_ij (dP_ij - delta_i)
+ *                        dQ_i  = scale sum_j dS_ij K_j
+ *                        dK_j += scale dS_ij Q_i,  dV_j += P_ij dO_i
+ * dK, dV accumulate over the query heads of a KV head.  Rows without a visible
+ * key contribute nothing (their dQ row is 0).  All arrays row-major; dQ like Q,
+ * dK / dV like K.  Returns 0, or -1 on bad arguments.
+ */
+int oracle_attn_bwd(double *dQ, double *dK, double *dV, const double *Q, const double *K,
+                    const double *V, const double *dO, int B, int Hq, int Hkv, int Sq, int Sk,
+                    int D, double scale, int causal, int window, int input_pos,
+                    const int *k_lengths, const int *q_lengths) {
+    if (B < 0 || Hq <= 0 || Hkv <= 0 || Sq < 0 || Sk < 0 || D <= 0) return -1;
+    if (Hq % Hkv != 0) return -1;
+    if (window > 0 && !causal) return -1;
+    const int group = Hq / Hkv;
+    memset(dQ, 0, sizeof(double) * (size_t)B * Hq * Sq * D);
+    memset(dK, 0, sizeof(double) * (size_t)B * Hkv * Sk * D);
+    memset(dV, 0, sizeof(double) * (size_t)B * Hkv * Sk * D);
+    int bad = 0;
+    /* one (b, KV head) per task: its dK / dV rows are written by this task only */
+#pragma omp parallel
+    {
+        double *prob = (double *)malloc(sizeof(double) * (Sk > 0 ? Sk : 1));
+        double *mrow = (double *)malloc(sizeof(double) * (Sk > 0 ? Sk : 1));
+        double *dpr = (double *)malloc(sizeof(double) * (Sk > 0 ? Sk : 1));
+        if (!prob || !mrow || !dpr) {
+#pragma omp atomic write
+            bad = 1;
+        }
+#pragma omp for schedule(dynamic, 1)
+        for (long bh = 0; bh < (long)B * Hkv; ++bh) {
+            if (!prob || !mrow || !dpr) continue;
+            const long b = bh / Hkv, hkv = bh % Hkv;
+            const int k_len = k_lengths ? k_lengths[b] : Sk;
+            const int q_len = q_lengths ? q_lengths[b] : Sq;
+            const double *Kh = K + bh * (long)Sk * D, *Vh = V + bh * (long)Sk * D;
+            double *dKh = dK + bh * (long)Sk * D, *dVh = dV + bh * (long)Sk * D;
+            for (long hq = hkv * group; hq < (hkv + 1) * group; ++hq) {
+                for (long i = 0; i < Sq; ++i) {
+                    const double *q = Q + ((b * Hq + hq) * (long)Sq + i) * D;
+                    const double *go = dO + ((b * Hq + hq) * (long)Sq + i) * D;
+                    double *gq = dQ + ((b * Hq + hq) * (long)Sq + i) * D;
+                    mask_row(mrow, i, Sk, causal, window, input_pos, k_len, q_len);
+                    double mx = -INFINITY;
+                    for (long j = 0; j < Sk; ++j) {
+                        double dot = 0.0;
+                        for (int d = 0; d < D; ++d) dot += q[d] * Kh[j * D + d];
+                        prob[j] = scale * dot + mrow[j];
+                        if (prob[j] > mx) mx = prob[j];
+                    }
+                    if (mx == -INFINITY) continue;
+                    double l = 0.0;
+                    for (long j = 0; j < Sk; ++j) {
+                        prob[j] = exp(prob[j] - mx);
+                        l += prob[j];
+                    }
+                    double delta = 0.0;
+                    for (long j = 0; j < Sk; ++j) {
+                        prob[j] /= l;
+                        double dp = 0.0;
+                        for (int d = 0; d < D; ++d) dp += go[d] * Vh[j * D + d];
+                        dpr[j] = dp;
+                        delta += prob[j] * dp;
+                    }
+                    for (long j = 0; j < Sk; ++j) {
+                        if (prob[j] == 0.0) continue;
+                        const double ds = prob[j] * (dpr[j] - delta);
+                        for (int d = 0; d < D; ++d) {
+                            gq[d] += scale * ds * Kh[j * D + d];
+                            dKh[j * D + d] += scale * ds * q[d];
+                            dVh[j * D + d] += prob[j] * go[d];
+                        }
+                    }
+                }
+            }
+        }
+        free(prob);
+        free(mrow);
+        free(dpr);
+    }
+    return bad ? -1 : 0;
 }

@@ -565,6 +565,67 @@ def pin_block_sparse_attention(orc):
         assert np.max(np.abs(O2[:, :1, sl] - Ob)) < 1e-12 and np.max(np.abs(L2[:, :1, sl] - Lb)) < 1e-12
 
 
+# --------------------------------------------------------------------------------------
+# Tylo.jl "Primitives" page: ∇attention!
+# --------------------------------------------------------------------------------------
+
+def pin_bwd_finite_differences(orc):
+    """Every gradient element equals the central difference of the loss sum(O * dO)
+    through the forward oracle (causal with input_pos, a window, ragged lengths,
+    GQA), to 1e-6."""
+    rng = _rng(51)
+    B, Hq, Hkv, Sq, Sk, D = 2, 2, 1, 4, 6, 3
+    Q, K, V = rng.standard_normal((B, Hq, Sq, D)), rng.standard_normal((B, Hkv, Sk, D)), \
+        rng.standard_normal((B, Hkv, Sk, D))
+    dO = rng.standard_normal((B, Hq, Sq, D))
+    kl, ql = np.array([6, 4], np.int32), np.array([4, 3], np.int32)
+    for causal, window, ip in ((True, 0, 2), (True, 3, 1), (False, 0, 0)):
+        kw = dict(causal=causal, window=window, input_pos=ip, k_lengths=kl, q_lengths=ql)
+        dQ, dK, dV = orc.attn_bwd(Q, K, V, dO, 0.6, **kw)
+
+        def loss(Q_, K_, V_):
+            O, _ = orc.attn_fwd(Q_, K_, V_, 0.6, **kw)
+            return float((O * dO).sum())
+        h = 1e-6
+        for X, G, which in ((Q, dQ, 0), (K, dK, 1), (V, dV, 2)):
+            for idx in np.ndindex(X.shape):
+                Xp, Xm = X.copy(), X.copy()
+                Xp[idx] += h
+                Xm[idx] -= h
+                args_p = [Q, K, V]
+                args_m = [Q, K, V]
+                args_p[which], args_m[which] = Xp, Xm
+                fd = (loss(*args_p) - loss(*args_m)) / (2 * h)
+                assert abs(fd - G[idx]) < 1e-6, (causal, window, which, idx, fd, G[idx])
+
+
+def pin_bwd_gqa_and_uniform(orc):
+    """GQA: dK / dV of a KV head are the sums of the MHA gradients of its query heads
+    on repeated K / V, and dQ is unchanged.  K = 0: uniform weights 1/n_i over the
+    visible keys, so dV_j = sum over rows i that see j of dO_i / n_i and dQ = 0."""
+    rng = _rng(52)
+    B, Hq, Hkv, S, D = 1, 4, 2, 7, 5
+    Q, K, V = rng.standard_normal((B, Hq, S, D)), rng.standard_normal((B, Hkv, S, D)), \
+        rng.standard_normal((B, Hkv, S, D))
+    dO = rng.standard_normal((B, Hq, S, D))
+    dQ, dK, dV = orc.attn_bwd(Q, K, V, dO, 0.4, causal=True)
+    mQ, mK, mV = orc.attn_bwd(Q, np.repeat(K, 2, axis=1), np.repeat(V, 2, axis=1), dO, 0.4,
+                              causal=True)
+    assert np.max(np.abs(dQ - mQ)) < 1e-12
+    assert np.max(np.abs(dK - mK.reshape(B, Hkv, 2, S, D).sum(2))) < 1e-12
+    assert np.max(np.abs(dV - mV.reshape(B, Hkv, 2, S, D).sum(2))) < 1e-12
+    Kz = np.zeros_like(K)
+    dQ, dK, dV = orc.attn_bwd(Q, Kz, V, dO, 0.4, causal=True, input_pos=2)
+    assert np.max(np.abs(dQ)) < 1e-12
+    want = np.zeros_like(V)
+    for h in range(Hq):
+        for i in range(S):
+            n = i + 3  # keys 0 .. input_pos + i, capped by S
+            n = min(n, S)
+            want[0, h // 2, :n] += dO[0, h, i] / n
+    assert np.max(np.abs(dV - want)) < 1e-12
+
+
 PINS = [
     pin_causal_mask_shape_and_rows,
     pin_sliding_window_rows,
@@ -590,4 +651,6 @@ PINS = [
     pin_rbs_degenerate_and_gqa,
     pin_rbs_relative_mask_golden,
     pin_block_sparse_attention,
+    pin_bwd_finite_differences,
+    pin_bwd_gqa_and_uniform,
 ]

@@ -77,6 +77,15 @@ MUTANTS = {
     "mask_band_wide": ("(qb - k < diagonal) && (k - qb < diagonal)", "(qb - k <= diagonal) && (k - qb <= diagonal)"),
     "mask_no_rescue": ("(sr[k] >= mr + log(alpha_rescue)) || band", "band"),
     "block_keep_ignored": ("if (!kr[j / 64]) mask[j] = -INFINITY;", "if (0) mask[j] = -INFINITY;"),
+    "bwd_dq_scale": ("gq[d] += scale * ds * Kh[j * D + d];", "gq[d] += ds * Kh[j * D + d];"),
+    "bwd_delta_zero": ("delta += prob[j] * dp;", "delta += 0.0 * dp;"),
+    "bwd_unnormalised": ("prob[j] /= l;", "prob[j] /= 1.0;"),
+    "bwd_dk_from_do": ("dKh[j * D + d] += scale * ds * q[d];", "dKh[j * D + d] += scale * ds * go[d];"),
+    "bwd_dv_from_ds": ("dVh[j * D + d] += prob[j] * go[d];", "dVh[j * D + d] += ds * go[d];"),
+    "bwd_one_head_per_group": ("for (long hq = hkv * group; hq < (hkv + 1) * group; ++hq)",
+                               "for (long hq = hkv * group; hq < hkv * group + 1; ++hq)"),
+    "bwd_mask_ignored": ("mask_row(mrow, i, Sk, causal, window, input_pos, k_len, q_len);",
+                         "mask_row(mrow, i, Sk, 0, 0, input_pos, Sk, Sq);"),
 }
 
 
