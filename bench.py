@@ -457,6 +457,44 @@ def time_block_sparse(dev, steps, warmup, peak):
                          "frac": tf / peak, "kernel": "attn_fwd_kernel<128, flex, block list>"}}
 
 
+def time_backward(step, steps, warmup, peak):
+    """Backward row (attn_bwd) on the step's LLM causal prefill: the forward's O and
+    LSE are made once outside the timed region; CUDA events per launch.  TFLOP/s
+    counts the five algorithmic products (S, dP, dV, dK, dQ): 2.5x the forward's
+    4 * D * visible pairs."""
+    from gqa_attention_flash_b200 import binding
+    w = step.pw
+    step.prefill()
+    dO = torch.randn(step.Q.shape, generator=torch.Generator().manual_seed(12)).to(
+        torch.bfloat16).to(step.dev)
+    dQ, dK, dV = torch.empty_like(step.Q), torch.empty_like(step.K), torch.empty_like(step.V)
+
+    def run():
+        binding.attn_bwd(dQ, dK, dV, dO, step.Q, step.K, step.V, step.O, step.LSE, w.scale,
+                         w.causal, w.window, w.input_pos, step.kl)
+    for _ in range(warmup):
+        run()
+    torch.cuda.synchronize()
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+          for _ in range(steps)]
+    for e0, e1 in ev:
+        e0.record()
+        run()
+        e1.record()
+    torch.cuda.synchronize()
+    st = binding.last_device_status()
+    if st != 0:
+        raise RuntimeError(f"backward device status: {binding.status_string(st)}")
+    ms = sum(a.elapsed_time(b) for a, b in ev) / steps
+    flops = 2.5 * step.prefill_flops
+    tf = flops / (ms * 1e-3) / 1e12
+    return {"workload": w.name + ", backward", "value": tf, "unit": "TFLOP/s",
+            "ms_per_launch": ms, "flops_per_launch": flops, "launches": steps,
+            "roofline": {"bound": "tensor", "achieved": tf, "peak": peak, "unit": "TFLOP/s",
+                         "frac": tf / peak,
+                         "kernel": "bwd_dkdv_kernel<128> + bwd_dq_kernel<128> + bwd_delta_kernel<128>"}}
+
+
 def time_paged(step, steps, warmup, peak):
     """Paged-KV decode row: the step's decode sequences scattered into a shuffled
     pool of 16-token blocks (block tables), device-resident; CUDA events around
@@ -585,9 +623,11 @@ def main(argv=None):
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-flex", action="store_true",
                     help="skip the flex_attention! measurements (reported apart from the step)")
+    ap.add_argument("--no-bwd", action="store_true",
+                    help="skip the backward measurement (reported apart from the step)")
     ap.add_argument("--no-paged", action="store_true",
                     help="skip the paged-KV decode measurement (reported apart from the step)")
-    ap.add_argument("--only", choices=["prefill", "decode", "flex", "paged"], default=None,
+    ap.add_argument("--only", choices=["prefill", "decode", "flex", "paged", "bwd"], default=None,
                     help="profiling: run one half of the step, or only the flex_attention! "
                          "workloads (no reported number)")
     ap.add_argument("--decode-batch", type=int, default=None,
@@ -615,6 +655,13 @@ def main(argv=None):
         pstep = Step(dev, "decode", args.decode_batch)
         res = time_paged(pstep, args.steps, args.warmup, peaks["hbm_gbs"])
         print(json.dumps({"profiling_run": True, "paged_ms": res["ms_per_launch"]}), flush=True)
+        return 0
+    if args.only == "bwd":
+        peaks, _ = load_peaks()
+        bstep = Step(dev, "prefill", None)
+        res = time_backward(bstep, args.steps, args.warmup, peaks["bf16_tflops"])
+        print(json.dumps({"profiling_run": True, "bwd_ms": res["ms_per_launch"],
+                          "bwd_tflops": res["value"]}), flush=True)
         return 0
     if args.only == "flex":
         peaks, _ = load_peaks()
@@ -695,6 +742,8 @@ def main(argv=None):
     if not args.no_flex:
         line["block_sparse"] = time_block_sparse(dev, min(K, 50), args.warmup,
                                                  peaks["bf16_tflops"])
+    if not args.no_bwd and step.do_prefill:
+        line["backward"] = time_backward(step, min(K, 30), args.warmup, peaks["bf16_tflops"])
     if not args.no_paged and step.do_decode:
         line["paged_decode"] = time_paged(step, min(K, 100), args.warmup, peaks["hbm_gbs"])
     print(json.dumps(line), flush=True)

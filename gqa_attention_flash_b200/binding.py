@@ -37,6 +37,8 @@ lib.attn_fwd_varlen.argtypes = [_p, _p, _p, _p, _p] + [_i] * 6 + [_f, _i, _i, _i
 lib.attn_fwd_flex.restype = _i
 lib.attn_fwd_flex.argtypes = [_p, _p, _p, _p, _p] + [_i] * 6 + [_f, _i, _i, _i, _p, _p, _f, _p, _p,
                                                                 _p, _p, _i, _p]
+lib.attn_bwd.restype = _i
+lib.attn_bwd.argtypes = [_p] * 8 + [_p] + [_i] * 6 + [_f, _i, _i, _i, _p, _p, _p]
 lib.attn_rbs_block_mask.restype = _i
 lib.attn_rbs_block_mask.argtypes = [_p, _p, _p, _p, _p] + [_i] * 6 + [_f, _f, _i, _p]
 _KEEP = ctypes.CFUNCTYPE(_i, _i, _i, _p)
@@ -135,6 +137,18 @@ def rbs_block_mask(Q, K, alpha_base=0.22, alpha_rescue=0.18, diagonal=1, want_sc
                                  int(diagonal), _stream(stream))
     _check(rc, "attn_rbs_block_mask")
     return (mask, base, resc) if want_scores else mask
+
+
+def attn_bwd(dQ, dK, dV, dO, Q, K, V, O, LSE, scale, causal=False, window=0, input_pos=0,
+             k_lengths=None, q_lengths=None, stream=None):
+    """Backward of attn_fwd: fill dQ (like Q) and dK, dV (like K, V) in place from dO,
+    the forward's inputs, output O and LSE."""
+    B, Hq, Sq, D = Q.shape
+    _, Hkv, Sk, _ = K.shape
+    rc = lib.attn_bwd(_ptr(dQ), _ptr(dK), _ptr(dV), _ptr(dO), _ptr(Q), _ptr(K), _ptr(V), _ptr(O),
+                      _ptr(LSE), B, Hq, Hkv, Sq, Sk, D, float(scale), int(causal), int(window),
+                      int(input_pos), _ptr(k_lengths), _ptr(q_lengths), _stream(stream))
+    _check(rc, "attn_bwd")
 
 
 def block_mask_shape(Sq: int, Sk: int):

@@ -278,6 +278,60 @@ attn_status_t attn_decode(void *O, const void *Q, const void *K, const void *V,
     return st;
 }
 
+attn_status_t attn_bwd(void *dQ, void *dK, void *dV, const void *dO, const void *Q, const void *K,
+                       const void *V, const void *O, const float *LSE, int B, int Hq, int Hkv,
+                       int Sq, int Sk, int D, float scale, int causal, int window, int input_pos,
+                       const int32_t *k_lengths, const int32_t *q_lengths, void *stream) {
+    attn_status_t st =
+        validate_fwd(const_cast<void *>(O), Q, K, V, nullptr, B, Hq, Hkv, Sq, Sk, D, scale, causal,
+                     window, input_pos);
+    if (st != ATTN_OK) return st;
+    const long long rows_q = (long long)B * Hq * Sq, rows_k = (long long)B * Hkv * Sk;
+    if (rows_q > 0 && (!dQ || !dO || !LSE)) return ATTN_ERR_NULL;
+    if (rows_k > 0 && (!dK || !dV)) return ATTN_ERR_NULL;
+    if (!aligned16(dQ) || !aligned16(dK) || !aligned16(dV) || !aligned16(dO) ||
+        (reinterpret_cast<uintptr_t>(LSE) & 3u))
+        return ATTN_ERR_INVALID;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    if (rows_q == 0) {  // no query: dK = dV = 0
+        if (rows_k > 0) {
+            const size_t bytes = (size_t)rows_k * D * 2;
+            if (cudaMemsetAsync(dK, 0, bytes, s) != cudaSuccess ||
+                cudaMemsetAsync(dV, 0, bytes, s) != cudaSuccess)
+                return ATTN_ERR_CUDA;
+        }
+        return ATTN_OK;
+    }
+    void *ws = nullptr;
+    if (cudaMallocAsync(&ws, (size_t)rows_q * sizeof(float), s) != cudaSuccess) return ATTN_ERR_CUDA;
+    BwdArgs a;
+    a.dQ = dQ;
+    a.dK = dK;
+    a.dV = dV;
+    a.dO = dO;
+    a.Q = Q;
+    a.K = K;
+    a.V = V;
+    a.O = O;
+    a.LSE = LSE;
+    a.k_lengths = k_lengths;
+    a.q_lengths = q_lengths;
+    a.B = B;
+    a.Hq = Hq;
+    a.Hkv = Hkv;
+    a.Sq = Sq;
+    a.Sk = Sk;
+    a.D = D;
+    a.scale = scale;
+    a.causal = causal;
+    a.window = window;
+    a.input_pos = input_pos;
+    a.delta = static_cast<float *>(ws);
+    st = launch_bwd(a, s);
+    if (cudaFreeAsync(ws, s) != cudaSuccess && st == ATTN_OK) st = ATTN_ERR_CUDA;
+    return st;
+}
+
 attn_status_t attn_rbs_block_mask(uint8_t *block_mask, float *base_scores, float *rescue_scores,
                                   const void *Q, const void *K, int B, int Hq, int Hkv, int Sq,
                                   int Sk, int D, float alpha_base, float alpha_rescue,

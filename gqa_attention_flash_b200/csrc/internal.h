@@ -54,6 +54,20 @@ struct DecodeArgs {
     int num_blocks = 0, block_size = 0, max_blocks = 0;
 };
 
+// Backward of the forward (Tylo.jl `∇attention!`).
+struct BwdArgs {
+    void *dQ, *dK, *dV;
+    const void *dO, *Q, *K, *V, *O;
+    const float *LSE;
+    const int32_t *k_lengths, *q_lengths;
+    int B, Hq, Hkv, Sq, Sk, D;
+    float scale;
+    int causal, window, input_pos;
+    float *delta;  // workspace (B, Hq, Sq)
+};
+
+attn_status_t launch_bwd(const BwdArgs &a, cudaStream_t stream);
+
 // Block scores + block mask of block-sparse prefill (RBS page of mlx-arsenal).
 struct RbsArgs {
     const void *Q, *K;

@@ -134,6 +134,28 @@ attn_status_t attn_fwd_flex(void *O, const void *Q, const void *K, const void *V
                             const uint8_t *block_mask, int block_mask_per_head, void *stream);
 
 /*
+ * attn_bwd -- backward of attn_fwd_varlen (Tylo.jl "Primitives" page, entry
+ * `∇attention!`: from the output gradient, the inputs, the output and the
+ * forward's saved softmax statistics, write the input gradients; overwrite).
+ *
+ *   dQ  [out] bf16 (B, Hq, Sq, D);  dK, dV [out] bf16 (B, Hkv, Sk, D)
+ *   dO  [in]  bf16 (B, Hq, Sq, D), the output gradient
+ *   Q, K, V, O [in] the forward's inputs and output
+ *   LSE [in]  float32 (B, Hq, Sq) saved by the forward (LSE = M + ln L)
+ *   scale, causal, window, input_pos, k_lengths, q_lengths: as in the forward
+ *   (they must match it).
+ * With P = exp(scale Q K^T - LSE) on the visible pairs: dV = P^T dO,
+ * dS = P (dO V^T - rowsum(dO O)), dQ = scale dS K, dK = scale dS^T Q; dK / dV
+ * of a KV head sum over the query heads it serves; keys never visible and
+ * query rows past q_lengths get zero gradients.  Allocates a stream-ordered
+ * workspace of B * Hq * Sq floats.  Errors as attn_fwd.
+ */
+attn_status_t attn_bwd(void *dQ, void *dK, void *dV, const void *dO, const void *Q, const void *K,
+                       const void *V, const void *O, const float *LSE, int B, int Hq, int Hkv,
+                       int Sq, int Sk, int D, float scale, int causal, int window, int input_pos,
+                       const int32_t *k_lengths, const int32_t *q_lengths, void *stream);
+
+/*
  * attn_rbs_block_mask -- block scores and block mask of block-sparse prefill
  * (mlx-arsenal "Radius-bounded block scores (RBS)" page: the block estimator of
  * "The idea", radius_bounded_block_scores and relative_block_mask of "What

@@ -1,0 +1,116 @@
+"""Attention backward on the GPU (attn_bwd through the C ABI, after attn_fwd_varlen
+on the GPU saved O and LSE) against the fp64 oracle's gradients from the
+definition, on the same seeded bf16 Q, K, V, dO.
+
+Tolerance (derived, the pages give none): the GPU rounds P and dS to bf16 before
+their second products and reads the bf16 output O for rowsum(dO O); each rounding
+is a relative 2^-9 on terms that add with mixed signs, so per tensor
+max |g_gpu - g_ref| <= 1e-2 * max |g_ref| + 1e-3."""
+import math
+
+import numpy as np
+import pytest
+import torch
+
+from gqa_attention_flash_b200 import workloads as W
+
+pytestmark = pytest.mark.gpu
+
+
+def gpu_fwd_bwd(Q, K, V, dO, scale, causal=False, window=0, input_pos=0, kl=None, ql=None):
+    from gqa_attention_flash_b200 import binding
+    dev = torch.device("cuda")
+    Qd, Kd, Vd, dOd = Q.to(dev), K.to(dev), V.to(dev), dO.to(dev)
+    O = torch.empty_like(Qd)
+    L = torch.empty(Q.shape[:3], dtype=torch.float32, device=dev)
+    kld = kl.to(dev) if kl is not None else None
+    qld = ql.to(dev) if ql is not None else None
+    binding.attn_fwd(O, Qd, Kd, Vd, L, scale, causal, window, input_pos, kld, qld)
+    dQ = torch.full_like(Qd, float("nan"))
+    dK = torch.full_like(Kd, float("nan"))
+    dV = torch.full_like(Vd, float("nan"))
+    binding.attn_bwd(dQ, dK, dV, dOd, Qd, Kd, Vd, O, L, scale, causal, window, input_pos, kld, qld)
+    st = binding.last_device_status()
+    assert st == 0, binding.status_string(st)
+    return dQ.cpu(), dK.cpu(), dV.cpu()
+
+
+def check(gpu, ref, what):
+    g = gpu.double().numpy()
+    assert np.all(np.isfinite(g)), f"{what}: non-finite"
+    tol = 1e-2 * float(np.abs(ref).max()) + 1e-3
+    err = float(np.abs(g - ref).max())
+    assert err <= tol, f"{what}: max err {err} > {tol}"
+    return err
+
+
+CASES = [
+    # B, Hq, Hkv, Sq, Sk, D, causal, window, input_pos, ragged
+    (1, 2, 2, 128, 128, 64, True, 0, 0, False),
+    (1, 4, 1, 200, 200, 128, True, 0, 0, False),
+    (2, 4, 2, 150, 333, 128, False, 0, 0, False),
+    (2, 2, 1, 100, 300, 64, True, 0, 200, False),
+    (1, 8, 2, 260, 260, 128, True, 70, 0, False),
+    (3, 4, 2, 190, 190, 128, True, 0, 0, True),
+]
+
+
+@pytest.mark.parametrize("case", CASES, ids=[str(c) for c in CASES])
+def test_backward_matches_oracle(orc, case):
+    B, Hq, Hkv, Sq, Sk, D, causal, window, ip, ragged = case
+    Q, K, V = W.random_prefill(70 + CASES.index(case), B, Hq, Hkv, Sq, Sk, D)
+    dO = torch.randn(B, Hq, Sq, D, generator=torch.Generator().manual_seed(5)).to(torch.bfloat16)
+    kl = ql = None
+    if ragged:
+        g = torch.Generator().manual_seed(8)
+        kl = torch.randint(0, Sk + 1, (B,), generator=g).to(torch.int32)
+        ql = torch.randint(1, Sq + 1, (B,), generator=g).to(torch.int32)
+    scale = 1.0 / math.sqrt(D)
+    dQ, dK, dV = gpu_fwd_bwd(Q, K, V, dO, scale, causal, window, ip, kl, ql)
+    rQ, rK, rV = orc.attn_bwd(Q.double().numpy(), K.double().numpy(), V.double().numpy(),
+                              dO.double().numpy(), scale, causal=causal, window=window,
+                              input_pos=ip, k_lengths=None if kl is None else kl.numpy(),
+                              q_lengths=None if ql is None else ql.numpy())
+    check(dQ, rQ, f"dQ {case}")
+    check(dK, rK, f"dK {case}")
+    check(dV, rV, f"dV {case}")
+
+
+def test_backward_masked_rows_and_keys_are_zero():
+    """Keys past k_len and rows past q_len get exactly zero gradients."""
+    B, Hq, Hkv, S, D = 2, 2, 1, 200, 128
+    Q, K, V = W.random_prefill(3, B, Hq, Hkv, S, S, D)
+    dO = torch.randn(B, Hq, S, D, generator=torch.Generator().manual_seed(2)).to(torch.bfloat16)
+    kl = torch.tensor([150, 0], dtype=torch.int32)
+    ql = torch.tensor([90, 200], dtype=torch.int32)
+    dQ, dK, dV = gpu_fwd_bwd(Q, K, V, dO, 0.1, True, 0, 0, kl, ql)
+    assert torch.all(dK[0, :, 150:] == 0) and torch.all(dV[0, :, 150:] == 0)
+    assert torch.all(dK[1] == 0) and torch.all(dV[1] == 0) and torch.all(dQ[1] == 0)
+    assert torch.all(dQ[0, :, 90:] == 0)
+
+
+def test_backward_full_size_llm(orc):
+    """The LLM causal shape (B4 Hq32 Hkv8 S4096 D128) as the benchmark runs it:
+    dQ on sampled rows and dK / dV on sampled keys of one batch entry, against the
+    oracle on a reduced problem that has exactly the same gradients there (the
+    first 512 queries of batch 0 see only keys < 512 under the causal mask)."""
+    w = W.LLM
+    x = W.make_prefill(w)
+    dO = torch.randn(x.Q.shape, generator=torch.Generator().manual_seed(11)).to(torch.bfloat16)
+    dQ, dK, dV = gpu_fwd_bwd(x.Q, x.K, x.V, dO, w.scale, True, 0, 0, x.k_lengths, None)
+    # rows < 512 of batch 0 depend only on keys < 512; keys < 512 collect gradients from every
+    # row, so compare dQ rows < 512 and dK / dV only through the reduced problem's dQ
+    n = 512
+    Qs, Ks, Vs, dOs = (t[:1, :, :n] for t in (x.Q, x.K, x.V, dO))
+    rQ, _, _ = orc.attn_bwd(Qs.double().numpy(), Ks.double().numpy(), Vs.double().numpy(),
+                            dOs.double().numpy(), w.scale, causal=True)
+    check(dQ[:1, :, :n], rQ, "full-size dQ rows < 512")
+    # the last key tile of batch 3 is seen only by the last rows: a reduced problem of rows
+    # [S - 128, S) against all keys gives the exact dK / dV of keys >= S - 128
+    m = 128
+    Qt, dOt = x.Q[3:4, :, -m:], dO[3:4, :, -m:]
+    _, rK, rV = orc.attn_bwd(Qt.double().numpy(), x.K[3:4].double().numpy(),
+                             x.V[3:4].double().numpy(), dOt.double().numpy(), w.scale,
+                             causal=True, input_pos=w.Sq - m)
+    check(dK[3:4, :, -m:], rK[:, :, -m:], "full-size dK keys >= S-128")
+    check(dV[3:4, :, -m:], rV[:, :, -m:], "full-size dV keys >= S-128")
