@@ -71,6 +71,38 @@ __device__ __forceinline__ void load_tile(uint8_t *dst, const __nv_bfloat16 *src
     }
 }
 
+// Asynchronous 16-byte global -> shared copies (zero-filled when `valid` is false;
+// the source address is then only a placeholder inside the tensor).
+__device__ __forceinline__ void cp_async16(uint32_t dst, const void *src, bool valid) {
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(dst), "l"(src),
+                 "r"(valid ? 16 : 0)
+                 : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+template <int N>
+__device__ __forceinline__ void cp_async_wait() {
+    asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
+}
+
+// load_tile with cp.async: rows [r0, r0 + 64) into the swizzled tile at `dst`.
+template <int D>
+__device__ __forceinline__ void load_tile_async(uint32_t dst, const __nv_bfloat16 *src, int r0,
+                                                int n_rows) {
+    constexpr int CH = D / 8;
+    for (int idx = threadIdx.x; idx < kT * CH; idx += kThreadsBwd) {
+        const int row = idx / CH, c = idx % CH;
+        const bool ok = r0 + row < n_rows;
+        cp_async16(dst + swz(row, c), src + (long long)(ok ? r0 + row : 0) * D + c * 8, ok);
+    }
+}
+
+// Asynchronous 4-byte copy (zero-filled when `valid` is false).
+__device__ __forceinline__ void cp_async4(uint32_t dst, const void *src, bool valid) {
+    asm volatile("cp.async.ca.shared.global [%0], [%1], 4, %2;" ::"r"(dst), "l"(src),
+                 "r"(valid ? 4 : 0)
+                 : "memory");
+}
+
 // Lengths of batch entry b, clamped to the tensor (a length past it is flagged).
 __device__ __forceinline__ void bwd_lengths(const BwdParams &p, int b, int &k_end, int &q_end) {
     k_end = p.Sk;
@@ -155,12 +187,14 @@ __device__ __forceinline__ void c_to_a(uint32_t (&a)[4], const float (&lo)[4], c
 template <int D>
 struct BwdCfg {
     static constexpr int TILE = kT * D * 2;  // bytes of one 64-row tile
-    static constexpr int OFF_A = 0;          // K (dkdv) or Q (dq)
-    static constexpr int OFF_B = TILE;       // V or dO
-    static constexpr int OFF_C = 2 * TILE;   // Q or K
-    static constexpr int OFF_D = 3 * TILE;   // dO or V
-    static constexpr int OFF_ROW = 4 * TILE; // 64 lse (log2 units) + 64 delta floats
-    static constexpr int SMEM = OFF_ROW + 2 * kT * 4 + 1024;
+    static constexpr int OFF_A = 0;          // K (dkdv) or Q (dq), resident
+    static constexpr int OFF_B = TILE;       // V or dO, resident
+    // two stages of streamed tiles: Q and dO (dkdv) or K and V (dq), then 64 LSE
+    // and 64 delta floats (dkdv)
+    static constexpr int STAGE = 2 * TILE + 2 * kT * 4;
+    static constexpr int OFF_S = 2 * TILE;
+    __host__ __device__ static constexpr int stage(int s) { return OFF_S + s * STAGE; }
+    static constexpr int SMEM = OFF_S + 2 * STAGE + 1024;
 };
 
 // ---------------------------------------------------------------------------------
@@ -174,8 +208,6 @@ __global__ void __launch_bounds__(kThreadsBwd, 1) bwd_dkdv_kernel(const BwdParam
     uint8_t *smem = reinterpret_cast<uint8_t *>(
         (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     const uint32_t sb = smem_u32(smem);
-    float *lse_s = reinterpret_cast<float *>(smem + C::OFF_ROW);
-    float *del_s = lse_s + kT;
     const int kt = blockIdx.x, hkv = blockIdx.y, b = blockIdx.z;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int g = lane >> 2, t = lane & 3;
@@ -200,19 +232,39 @@ __global__ void __launch_bounds__(kThreadsBwd, 1) bwd_dkdv_kernel(const BwdParam
     if (p.window > 0) i_hi = min(i_hi, kv0 + kT + p.window - p.input_pos);
     const int qt_lo = i_lo / kT, qt_hi = i_hi > i_lo ? (i_hi + kT - 1) / kT : qt_lo;
 
-    for (int hq = hkv * p.group; hq < (hkv + 1) * p.group; ++hq) {
-        const long long q_base = (long long)(b * p.Hq + hq) * p.Sq;
-        for (int qt = qt_lo; qt < qt_hi; ++qt) {
-            const int q0 = qt * kT;
-            __syncthreads();  // the previous tile's reads are done
-            load_tile<D>(smem + C::OFF_C, p.Q + q_base * D, q0, p.Sq);
-            load_tile<D>(smem + C::OFF_D, p.dO + q_base * D, q0, p.Sq);
-            if (threadIdx.x < kT) {
-                const int i = q0 + threadIdx.x;
-                lse_s[threadIdx.x] = i < p.Sq ? p.LSE[q_base + i] * 1.4426950408889634f : 0.f;
-                del_s[threadIdx.x] = i < p.Sq ? p.delta[q_base + i] : 0.f;
-            }
+    // (query head, query tile) pairs in order, the next one's Q, dO, LSE and delta
+    // copied asynchronously into the other stage while this one is computed
+    const int n_qt = qt_hi - qt_lo;
+    const int n_it = p.group * n_qt;
+    auto issue = [&](int it) {
+        const int hq = hkv * p.group + it / n_qt;
+        const int q0 = (qt_lo + it % n_qt) * kT;
+        const long long qb = (long long)(b * p.Hq + hq) * p.Sq;
+        const uint32_t st = sb + C::stage(it & 1);
+        load_tile_async<D>(st, p.Q + qb * D, q0, p.Sq);
+        load_tile_async<D>(st + C::TILE, p.dO + qb * D, q0, p.Sq);
+        if (threadIdx.x < kT) {
+            const int i = q0 + threadIdx.x;
+            const bool ok = i < p.Sq;
+            cp_async4(st + 2 * C::TILE + 4 * threadIdx.x, p.LSE + qb + (ok ? i : 0), ok);
+            cp_async4(st + 2 * C::TILE + 4 * (kT + threadIdx.x), p.delta + qb + (ok ? i : 0), ok);
+        }
+        cp_async_commit();
+    };
+    if (n_it > 0) issue(0);
+    for (int it = 0; it < n_it; ++it) {
+        {
+            if (it + 1 < n_it)
+                issue(it + 1);
+            else
+                cp_async_commit();  // empty group: the wait below always leaves one pending
+            cp_async_wait<1>();
             __syncthreads();
+            const int q0 = (qt_lo + it % n_qt) * kT;
+            const uint32_t so = C::stage(it & 1);
+            const uint32_t tq = sb + so, tdo = sb + so + C::TILE;
+            const float *lse_s = reinterpret_cast<const float *>(smem + so + 2 * C::TILE);
+            const float *del_s = lse_s + kT;
 
             // S^T (16 keys of this warp x 64 queries)
             float st[8][4];
@@ -225,7 +277,7 @@ __global__ void __launch_bounds__(kThreadsBwd, 1) bwd_dkdv_kernel(const BwdParam
 #pragma unroll
                 for (int np = 0; np < 4; ++np) {
                     uint32_t bq[4];
-                    ld_b_rows(bq, sb + C::OFF_C, np * 16, kk, lane);
+                    ld_b_rows(bq, tq, np * 16, kk, lane);
                     mma_m16n8k16(st[2 * np], a, bq[0], bq[1]);
                     mma_m16n8k16(st[2 * np + 1], a, bq[2], bq[3]);
                 }
@@ -237,7 +289,7 @@ __global__ void __launch_bounds__(kThreadsBwd, 1) bwd_dkdv_kernel(const BwdParam
                 for (int e = 0; e < 4; ++e) {
                     const int j = kv0 + warp * 16 + g + (e >> 1) * 8;
                     const int il = n * 8 + 2 * t + (e & 1);
-                    const float lse = lse_s[il];
+                    const float lse = lse_s[il] * 1.4426950408889634f;
                     const bool vis = visible(p, q0 + il, j, k_end, q_end) && lse != neg_inf();
                     st[n][e] = vis ? fast_exp2(fmaf(st[n][e], p.scale_log2, -lse)) : 0.f;
                 }
@@ -249,7 +301,7 @@ __global__ void __launch_bounds__(kThreadsBwd, 1) bwd_dkdv_kernel(const BwdParam
 #pragma unroll
                 for (int dp = 0; dp < D / 16; ++dp) {
                     uint32_t bo[4];
-                    ld_b_cols(bo, sb + C::OFF_D, kq * 16, dp, lane);
+                    ld_b_cols(bo, tdo, kq * 16, dp, lane);
                     mma_m16n8k16(dv[2 * dp], a, bo[0], bo[1]);
                     mma_m16n8k16(dv[2 * dp + 1], a, bo[2], bo[3]);
                 }
@@ -265,7 +317,7 @@ __global__ void __launch_bounds__(kThreadsBwd, 1) bwd_dkdv_kernel(const BwdParam
 #pragma unroll
                 for (int np = 0; np < 4; ++np) {
                     uint32_t bq[4];
-                    ld_b_rows(bq, sb + C::OFF_D, np * 16, kk, lane);
+                    ld_b_rows(bq, tdo, np * 16, kk, lane);
                     mma_m16n8k16(dpt[2 * np], a, bq[0], bq[1]);
                     mma_m16n8k16(dpt[2 * np + 1], a, bq[2], bq[3]);
                 }
@@ -283,13 +335,15 @@ __global__ void __launch_bounds__(kThreadsBwd, 1) bwd_dkdv_kernel(const BwdParam
 #pragma unroll
                 for (int dp = 0; dp < D / 16; ++dp) {
                     uint32_t bq[4];
-                    ld_b_cols(bq, sb + C::OFF_C, kq * 16, dp, lane);
+                    ld_b_cols(bq, tq, kq * 16, dp, lane);
                     mma_m16n8k16(dk[2 * dp], a, bq[0], bq[1]);
                     mma_m16n8k16(dk[2 * dp + 1], a, bq[2], bq[3]);
                 }
             }
         }
+        __syncthreads();  // every warp is done with this stage before it is refilled
     }
+    cp_async_wait<0>();
     // write dK (scaled) and dV rows of this warp's 16 keys
 #pragma unroll
     for (int half = 0; half < 2; ++half) {
@@ -356,12 +410,24 @@ __global__ void __launch_bounds__(kThreadsBwd, 1) bwd_dq_kernel(const BwdParams 
             hi = static_cast<int>((h + kT - 1) / kT);
         }
     }
+    // key tiles in order, the next one's K and V copied asynchronously into the
+    // other stage while this one is computed
+    auto issue = [&](int kt) {
+        const uint32_t st = sb + C::stage((kt - lo) & 1);
+        load_tile_async<D>(st, p.K + kv_base * D, kt * kT, p.Sk);
+        load_tile_async<D>(st + C::TILE, p.V + kv_base * D, kt * kT, p.Sk);
+        cp_async_commit();
+    };
+    if (hi > lo) issue(lo);
     for (int kt = lo; kt < hi; ++kt) {
         const int kv0 = kt * kT;
+        if (kt + 1 < hi)
+            issue(kt + 1);
+        else
+            cp_async_commit();  // empty group: the wait below always leaves one pending
+        cp_async_wait<1>();
         __syncthreads();
-        load_tile<D>(smem + C::OFF_C, p.K + kv_base * D, kv0, p.Sk);
-        load_tile<D>(smem + C::OFF_D, p.V + kv_base * D, kv0, p.Sk);
-        __syncthreads();
+        const uint32_t tk = sb + C::stage((kt - lo) & 1), tv = tk + C::TILE;
         // S (16 rows of this warp x 64 keys)
         float s[8][4];
 #pragma unroll
@@ -373,7 +439,7 @@ __global__ void __launch_bounds__(kThreadsBwd, 1) bwd_dq_kernel(const BwdParams 
 #pragma unroll
             for (int np = 0; np < 4; ++np) {
                 uint32_t bk[4];
-                ld_b_rows(bk, sb + C::OFF_C, np * 16, kk, lane);
+                ld_b_rows(bk, tk, np * 16, kk, lane);
                 mma_m16n8k16(s[2 * np], a, bk[0], bk[1]);
                 mma_m16n8k16(s[2 * np + 1], a, bk[2], bk[3]);
             }
@@ -399,7 +465,7 @@ __global__ void __launch_bounds__(kThreadsBwd, 1) bwd_dq_kernel(const BwdParams 
 #pragma unroll
             for (int np = 0; np < 4; ++np) {
                 uint32_t bv[4];
-                ld_b_rows(bv, sb + C::OFF_D, np * 16, kk, lane);
+                ld_b_rows(bv, tv, np * 16, kk, lane);
                 mma_m16n8k16(dps[2 * np], a, bv[0], bv[1]);
                 mma_m16n8k16(dps[2 * np + 1], a, bv[2], bv[3]);
             }
@@ -416,12 +482,14 @@ __global__ void __launch_bounds__(kThreadsBwd, 1) bwd_dq_kernel(const BwdParams 
 #pragma unroll
             for (int dp = 0; dp < D / 16; ++dp) {
                 uint32_t bk[4];
-                ld_b_cols(bk, sb + C::OFF_C, kq * 16, dp, lane);
+                ld_b_cols(bk, tk, kq * 16, dp, lane);
                 mma_m16n8k16(dq[2 * dp], a, bk[0], bk[1]);
                 mma_m16n8k16(dq[2 * dp + 1], a, bk[2], bk[3]);
             }
         }
+        __syncthreads();  // every warp is done with this stage before it is refilled
     }
+    cp_async_wait<0>();
 #pragma unroll
     for (int half = 0; half < 2; ++half) {
         const int i = q0 + warp * 16 + g + half * 8;
