@@ -543,12 +543,7 @@ attn_status_t launch_bwd_d(const BwdArgs &a, cudaStream_t stream) {
     const long long rows = (long long)a.B * a.Hq * a.Sq;
     bwd_delta_kernel<D><<<static_cast<unsigned>((rows + 7) / 8), 256, 0, stream>>>(p, rows);
     if (cudaGetLastError() != cudaSuccess) return ATTN_ERR_CUDA;
-    if (a.Sk > 0) {
-        bwd_dkdv_kernel<D><<<dim3((a.Sk + kT - 1) / kT, a.Hkv, a.B), kThreadsBwd, C::SMEM, stream>>>(p);
-        if (cudaGetLastError() != cudaSuccess) return ATTN_ERR_CUDA;
-    }
-    bwd_dq_kernel<D><<<dim3((a.Sq + kT - 1) / kT, a.Hq, a.B), kThreadsBwd, C::SMEM, stream>>>(p);
-    return cudaGetLastError() == cudaSuccess ? ATTN_OK : ATTN_ERR_CUDA;
+    return launch_bwd_tc(a, stream);
 }
 
 }  // namespace

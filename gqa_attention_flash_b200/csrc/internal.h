@@ -67,6 +67,8 @@ struct BwdArgs {
 };
 
 attn_status_t launch_bwd(const BwdArgs &a, cudaStream_t stream);
+// dK / dV and dQ on tcgen05 (after the delta workspace is written).
+attn_status_t launch_bwd_tc(const BwdArgs &a, cudaStream_t stream);
 
 // Block scores + block mask of block-sparse prefill (RBS page of mlx-arsenal).
 struct RbsArgs {
