@@ -56,10 +56,13 @@ struct TcCfg {
     static constexpr int OFF_S = 2 * TILE;
     __host__ __device__ static constexpr int stage(int s) { return OFF_S + s * STAGE; }
     static constexpr int OFF_BAR = OFF_S + NS * STAGE;
-    // barriers: resident, full[NS], empty[NS], s_full, dp_full, p_done, ds_full, done
-    static constexpr int BAR_RES = 0, BAR_FULL = 1, BAR_EMPTY = 1 + NS, BAR_SFULL = 1 + 2 * NS,
-                         BAR_DPFULL = 2 + 2 * NS, BAR_PDONE = 3 + 2 * NS, BAR_DSFULL = 4 + 2 * NS,
-                         BAR_DONE = 5 + 2 * NS, N_BARS = 6 + 2 * NS;
+    // barriers: resident; per ring slot full / empty of its Q half and of its dO
+    // half (they are released at different points); s_full, dp_full, p_done,
+    // ds_full, done
+    static constexpr int BAR_RES = 0, BAR_FULLQ = 1, BAR_EMPTYQ = 1 + NS, BAR_FULLD = 1 + 2 * NS,
+                         BAR_EMPTYD = 1 + 3 * NS, BAR_SFULL = 1 + 4 * NS, BAR_DPFULL = 2 + 4 * NS,
+                         BAR_PDONE = 3 + 4 * NS, BAR_DSFULL = 4 + 4 * NS, BAR_DONE = 5 + 4 * NS,
+                         N_BARS = 6 + 4 * NS;
     static constexpr int OFF_MISC = OFF_BAR + N_BARS * 8;
     static constexpr int SMEM = OFF_MISC + 16 + 1024;
     // TMEM columns
@@ -156,24 +159,16 @@ __device__ __forceinline__ void mma_tmem_a(uint32_t d_tmem, uint32_t a_tmem, uin
     }
 }
 
-// Shared set-up: barriers, TMEM allocation (warp 9), 512 columns.
-template <int D>
+// Shared set-up: barriers (the elementwise warps' arrival barriers count 256
+// arrivals, the others one), TMEM allocation (warp 9), 512 columns.
+template <class C>
 __device__ __forceinline__ uint32_t tc_setup(uint8_t *smem, uint32_t sbase) {
-    using C = TcCfg<D>;
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + C::OFF_MISC);
     volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + C::OFF_MISC + 4);
-    auto bar = [&](int i) -> uint32_t { return sbase + C::OFF_BAR + 8 * i; };
     if (threadIdx.x == 0) {
-        mbar_init(bar(C::BAR_RES), 1);
-        for (int s = 0; s < C::NS; ++s) {
-            mbar_init(bar(C::BAR_FULL + s), 1);
-            mbar_init(bar(C::BAR_EMPTY + s), 1);
-        }
-        mbar_init(bar(C::BAR_SFULL), 1);
-        mbar_init(bar(C::BAR_DPFULL), 1);
-        mbar_init(bar(C::BAR_PDONE), kEltThreads);
-        mbar_init(bar(C::BAR_DSFULL), kEltThreads);
-        mbar_init(bar(C::BAR_DONE), 1);
+        for (int i = 0; i < C::N_BARS; ++i)
+            mbar_init(sbase + C::OFF_BAR + 8 * i,
+                      (i == C::BAR_PDONE || i == C::BAR_DSFULL) ? kEltThreads : 1);
         *abort_flag = 0;
         fence_mbar_init();
     }
@@ -188,9 +183,8 @@ __device__ __forceinline__ uint32_t tc_setup(uint8_t *smem, uint32_t sbase) {
 }
 
 // Shared teardown: let work in flight land after a give-up, free TMEM.
-template <int D>
+template <class C>
 __device__ __forceinline__ void tc_teardown(uint8_t *smem, uint32_t tmem) {
-    using C = TcCfg<D>;
     volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + C::OFF_MISC + 4);
     if (*abort_flag) drain_delay(2000000);
     tc_fence_before();
@@ -241,6 +235,8 @@ __global__ void __launch_bounds__(kThreadsTc, 1)
                        const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmdO,
                        const TcParams p) {
     using C = TcCfg<D>;
+    // key tiles in increasing order, the (KV head, batch) pairs fastest: under a
+    // causal mask the heaviest tiles go first
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>(
         (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -248,7 +244,8 @@ __global__ void __launch_bounds__(kThreadsTc, 1)
     auto bar = [&](int i) -> uint32_t { return sbase + C::OFF_BAR + 8 * i; };
     volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + C::OFF_MISC + 4);
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int kt = blockIdx.x, hkv = blockIdx.y, b = blockIdx.z;
+    const int hkv = blockIdx.x % p.Hkv, b = (blockIdx.x / p.Hkv) % p.B,
+              kt = blockIdx.x / (p.Hkv * p.B);
     const int kv0 = kt * TB;
     int k_end, q_end;
     tc_lengths(p, b, k_end, q_end);
@@ -260,7 +257,7 @@ __global__ void __launch_bounds__(kThreadsTc, 1)
     const int qt_lo = i_lo / TB, qt_hi = i_hi > i_lo ? (i_hi + TB - 1) / TB : qt_lo;
     const int n_qt = qt_hi - qt_lo, n_it = p.group * n_qt;
 
-    const uint32_t tmem = tc_setup<D>(smem, sbase);
+    const uint32_t tmem = tc_setup<C>(smem, sbase);
 
     if (warp == kWarpTmaB) {
         // ===================== TMA producer =====================
@@ -280,28 +277,44 @@ __global__ void __launch_bounds__(kThreadsTc, 1)
             }
             for (int it = 0; it < n_it; ++it) {
                 const int st = it % C::NS, use = it / C::NS;
-                if (use > 0 && !warp_wait(bar(C::BAR_EMPTY + st), (use - 1) & 1, abort_flag,
-                                          p.wait_limit_ns, p.status))
-                    break;
                 const int hq = hkv * p.group + it / n_qt;
                 const int q0 = (qt_lo + it % n_qt) * TB;
                 const long long qrow = (long long)(b * p.Hq + hq) * p.Sq;
-                float *rows = reinterpret_cast<float *>(smem + C::stage(st) + 2 * C::TILE);
-                for (int r = lane; r < TB; r += 32) {  // LSE (log2 units) and delta of the tile
-                    const int i = q0 + r;
+                // the tile's LSE (log2 units) and delta, loaded before the slot is free
+                float lr[TB / 32], dr[TB / 32];
+#pragma unroll
+                for (int k = 0; k < TB / 32; ++k) {
+                    const int i = q0 + lane + 32 * k;
                     const bool ok = i < p.Sq;
-                    rows[r] = ok ? p.LSE[qrow + i] * kLog2e : ninf();
-                    rows[TB + r] = ok ? p.delta[qrow + i] : 0.f;
+                    lr[k] = ok ? p.LSE[qrow + i] * kLog2e : ninf();
+                    dr[k] = ok ? p.delta[qrow + i] : 0.f;
+                }
+                // dO half: free once dV of the slot's previous item has run
+                if (use > 0 && !warp_wait(bar(C::BAR_EMPTYD + st), (use - 1) & 1, abort_flag,
+                                          p.wait_limit_ns, p.status))
+                    break;
+                if (lane == 0) {
+                    mbar_arrive_expect_tx(bar(C::BAR_FULLD + st), C::TILE);
+                    for (int c = 0; c < C::NBOX; ++c)
+                        tma_load_3d(sbase + C::stage(st) + C::TILE + c * C::BOX, &tmdO,
+                                    bar(C::BAR_FULLD + st), c * 64, q0, b * p.Hq + hq);
+                }
+                // Q half and the rows: free once dK of the slot's previous item has run
+                if (use > 0 && !warp_wait(bar(C::BAR_EMPTYQ + st), (use - 1) & 1, abort_flag,
+                                          p.wait_limit_ns, p.status))
+                    break;
+                float *rows = reinterpret_cast<float *>(smem + C::stage(st) + 2 * C::TILE);
+#pragma unroll
+                for (int k = 0; k < TB / 32; ++k) {
+                    rows[lane + 32 * k] = lr[k];
+                    rows[TB + lane + 32 * k] = dr[k];
                 }
                 __syncwarp();
                 if (lane == 0) {
-                    mbar_arrive_expect_tx(bar(C::BAR_FULL + st), 2 * C::TILE);
-                    for (int c = 0; c < C::NBOX; ++c) {
-                        tma_load_3d(sbase + C::stage(st) + c * C::BOX, &tmQ, bar(C::BAR_FULL + st),
+                    mbar_arrive_expect_tx(bar(C::BAR_FULLQ + st), C::TILE);
+                    for (int c = 0; c < C::NBOX; ++c)
+                        tma_load_3d(sbase + C::stage(st) + c * C::BOX, &tmQ, bar(C::BAR_FULLQ + st),
                                     c * 64, q0, b * p.Hq + hq);
-                        tma_load_3d(sbase + C::stage(st) + C::TILE + c * C::BOX, &tmdO,
-                                    bar(C::BAR_FULL + st), c * 64, q0, b * p.Hq + hq);
-                    }
                 }
                 __syncwarp();
             }
@@ -310,7 +323,7 @@ __global__ void __launch_bounds__(kThreadsTc, 1)
         // ===================== MMA issuer =====================
         if (lane == 0 && n_it > 0) {
             bool ok = mbar_wait(bar(C::BAR_RES), 0, abort_flag, p.wait_limit_ns, p.status) &&
-                      mbar_wait(bar(C::BAR_FULL), 0, abort_flag, p.wait_limit_ns, p.status);
+                      mbar_wait(bar(C::BAR_FULLQ), 0, abort_flag, p.wait_limit_ns, p.status);
             if (ok) {
                 tc_fence_after();
                 mma_kmajor<D>(tmem + C::COL_S, sbase + C::OFF_R0, sbase + C::stage(0));  // S^T = K Q^T
@@ -319,15 +332,20 @@ __global__ void __launch_bounds__(kThreadsTc, 1)
             for (int it = 0; ok && it < n_it; ++it) {
                 const int st = it % C::NS;
                 const uint32_t q_s = sbase + C::stage(st), do_s = q_s + C::TILE;
+                if (!(ok = mbar_wait(bar(C::BAR_FULLD + st), (it / C::NS) & 1, abort_flag,
+                                     p.wait_limit_ns, p.status)))
+                    break;
+                tc_fence_after();
                 mma_kmajor<D>(tmem + C::COL_DP, sbase + C::OFF_R1, do_s);  // dP^T = V dO^T
                 mma_commit(bar(C::BAR_DPFULL));
                 if (!(ok = mbar_wait(bar(C::BAR_PDONE), it & 1, abort_flag, p.wait_limit_ns, p.status)))
                     break;
                 tc_fence_after();
                 mma_tmem_a<D, true>(tmem + C::COL_A, tmem + C::COL_S, do_s, it > 0);  // dV += P^T dO
+                mma_commit(bar(C::BAR_EMPTYD + st));
                 if (it + 1 < n_it) {
                     const int st1 = (it + 1) % C::NS;
-                    if (!(ok = mbar_wait(bar(C::BAR_FULL + st1), ((it + 1) / C::NS) & 1, abort_flag,
+                    if (!(ok = mbar_wait(bar(C::BAR_FULLQ + st1), ((it + 1) / C::NS) & 1, abort_flag,
                                          p.wait_limit_ns, p.status)))
                         break;
                     tc_fence_after();
@@ -338,7 +356,7 @@ __global__ void __launch_bounds__(kThreadsTc, 1)
                     break;
                 tc_fence_after();
                 mma_tmem_a<D, true>(tmem + C::COL_B, tmem + C::COL_DP, q_s, it > 0);  // dK += dS^T Q
-                mma_commit(bar(C::BAR_EMPTY + st));
+                mma_commit(bar(C::BAR_EMPTYQ + st));
             }
             if (ok) mma_commit(bar(C::BAR_DONE));
         }
@@ -355,7 +373,7 @@ __global__ void __launch_bounds__(kThreadsTc, 1)
             // S^T(it) in TMEM; the producer's plain stores of LSE / delta are
             // published by its arrive on the stage's full barrier
             if (!warp_wait(bar(C::BAR_SFULL), it & 1, abort_flag, p.wait_limit_ns, p.status) ||
-                !warp_wait(bar(C::BAR_FULL + st), (it / C::NS) & 1, abort_flag, p.wait_limit_ns,
+                !warp_wait(bar(C::BAR_FULLQ + st), (it / C::NS) & 1, abort_flag, p.wait_limit_ns,
                            p.status)) {
                 ok = false;
                 break;
@@ -445,18 +463,41 @@ __global__ void __launch_bounds__(kThreadsTc, 1)
             tc_zero_half<D>(p.dK + krow * D, half * (D / 2));
         }
     }
-    tc_teardown<D>(smem, tmem);
+    tc_teardown<C>(smem, tmem);
 }
 
 // ---------------------------------------------------------------------------------
 // dQ of one 128-row query tile
 // ---------------------------------------------------------------------------------
+// Shared memory of the dQ kernel: Q and dO resident, three K slots and two V
+// slots (K of a tile is read last, by dQ += dS K, and first, by the next-but-one
+// S, so it gets the deeper ring).
+template <int D>
+struct DqCfg {
+    static constexpr int NBOX = D / 64;
+    static constexpr int BOX = TB * 128;
+    static constexpr int TILE = TB * D * 2;
+    static constexpr int NK = 3, NV = 2;
+    static constexpr int OFF_Q = 0, OFF_DO = TILE;
+    __host__ __device__ static constexpr int k_slot(int s) { return 2 * TILE + s * TILE; }
+    __host__ __device__ static constexpr int v_slot(int s) { return (2 + NK) * TILE + s * TILE; }
+    static constexpr int OFF_BAR = (2 + NK + NV) * TILE;
+    static constexpr int BAR_RES = 0, BAR_FULLK = 1, BAR_EMPTYK = 1 + NK, BAR_FULLV = 1 + 2 * NK,
+                         BAR_EMPTYV = 1 + 2 * NK + NV, BAR_SFULL = 1 + 2 * NK + 2 * NV,  // two
+                         BAR_DPFULL = 3 + 2 * NK + 2 * NV, BAR_DSFULL = 4 + 2 * NK + 2 * NV,
+                         BAR_DONE = 5 + 2 * NK + 2 * NV, BAR_PDONE = -1, N_BARS = 6 + 2 * NK + 2 * NV;
+    static constexpr int OFF_MISC = OFF_BAR + N_BARS * 8;
+    static constexpr int SMEM = OFF_MISC + 16 + 1024;
+    // TMEM: two S buffers (dS written over its own S), dP, dQ
+    static constexpr uint32_t COL_S = 0, COL_DP = 2 * TB, COL_DQ = 3 * TB;
+};
+
 template <int D>
 __global__ void __launch_bounds__(kThreadsTc, 1)
     bwd_dq_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                      const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmdO,
                      const TcParams p, int n_qt_total) {
-    using C = TcCfg<D>;
+    using C = DqCfg<D>;
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>(
         (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -489,7 +530,7 @@ __global__ void __launch_bounds__(kThreadsTc, 1)
     }
     const int n_kt = hi - lo;
 
-    const uint32_t tmem = tc_setup<D>(smem, sbase);
+    const uint32_t tmem = tc_setup<C>(smem, sbase);
 
     if (warp == kWarpTmaB) {
         // ===================== TMA producer =====================
@@ -500,67 +541,72 @@ __global__ void __launch_bounds__(kThreadsTc, 1)
             prefetch_tensormap(&tmdO);
             mbar_arrive_expect_tx(bar(C::BAR_RES), 2 * C::TILE);
             for (int c = 0; c < C::NBOX; ++c) {
-                tma_load_3d(sbase + C::OFF_R0 + c * C::BOX, &tmQ, bar(C::BAR_RES), c * 64, q0,
+                tma_load_3d(sbase + C::OFF_Q + c * C::BOX, &tmQ, bar(C::BAR_RES), c * 64, q0,
                             b * p.Hq + hq);
-                tma_load_3d(sbase + C::OFF_R1 + c * C::BOX, &tmdO, bar(C::BAR_RES), c * 64, q0,
+                tma_load_3d(sbase + C::OFF_DO + c * C::BOX, &tmdO, bar(C::BAR_RES), c * 64, q0,
                             b * p.Hq + hq);
             }
             for (int g = 0; g < n_kt; ++g) {
-                const int st = g % C::NS, use = g / C::NS;
-                if (use > 0 && !mbar_wait(bar(C::BAR_EMPTY + st), (use - 1) & 1, abort_flag,
-                                          p.wait_limit_ns, p.status))
-                    break;
                 const int kv0 = (lo + g) * TB;
-                mbar_arrive_expect_tx(bar(C::BAR_FULL + st), 2 * C::TILE);
-                for (int c = 0; c < C::NBOX; ++c) {
-                    tma_load_3d(sbase + C::stage(st) + c * C::BOX, &tmK, bar(C::BAR_FULL + st), c * 64,
+                const int ks = g % C::NK, ku = g / C::NK, vs = g % C::NV, vu = g / C::NV;
+                if (ku > 0 && !mbar_wait(bar(C::BAR_EMPTYK + ks), (ku - 1) & 1, abort_flag,
+                                         p.wait_limit_ns, p.status))
+                    break;
+                mbar_arrive_expect_tx(bar(C::BAR_FULLK + ks), C::TILE);
+                for (int c = 0; c < C::NBOX; ++c)
+                    tma_load_3d(sbase + C::k_slot(ks) + c * C::BOX, &tmK, bar(C::BAR_FULLK + ks), c * 64,
                                 kv0, b * p.Hkv + hkv);
-                    tma_load_3d(sbase + C::stage(st) + C::TILE + c * C::BOX, &tmV,
-                                bar(C::BAR_FULL + st), c * 64, kv0, b * p.Hkv + hkv);
-                }
+                if (vu > 0 && !mbar_wait(bar(C::BAR_EMPTYV + vs), (vu - 1) & 1, abort_flag,
+                                         p.wait_limit_ns, p.status))
+                    break;
+                mbar_arrive_expect_tx(bar(C::BAR_FULLV + vs), C::TILE);
+                for (int c = 0; c < C::NBOX; ++c)
+                    tma_load_3d(sbase + C::v_slot(vs) + c * C::BOX, &tmV, bar(C::BAR_FULLV + vs), c * 64,
+                                kv0, b * p.Hkv + hkv);
             }
         }
     } else if (warp == kWarpMmaB) {
         // ===================== MMA issuer =====================
-        constexpr uint32_t COL_DS = C::COL_B;  // dS, bf16 pairs, 64 columns
+        // order: S(0), dP(0), S(1), then per tile g: [dS(g)] dQ += dS(g) K(g), dP(g+1),
+        // S(g+2) -- S(g+2) reuses the TMEM buffer of S(g) / dS(g) after dQ(g) read it
         if (lane == 0 && n_kt > 0) {
-            bool ok = mbar_wait(bar(C::BAR_RES), 0, abort_flag, p.wait_limit_ns, p.status) &&
-                      mbar_wait(bar(C::BAR_FULL), 0, abort_flag, p.wait_limit_ns, p.status);
-            if (ok) {
+            auto issue_s = [&](int g) -> bool {
+                const int ks = g % C::NK;
+                if (!mbar_wait(bar(C::BAR_FULLK + ks), (g / C::NK) & 1, abort_flag, p.wait_limit_ns,
+                               p.status))
+                    return false;
                 tc_fence_after();
-                const uint32_t k_s = sbase + C::stage(0);
-                mma_kmajor<D>(tmem + C::COL_S, sbase + C::OFF_R0, k_s);             // S = Q K^T
-                mma_commit(bar(C::BAR_SFULL));
-                mma_kmajor<D>(tmem + C::COL_DP, sbase + C::OFF_R1, k_s + C::TILE);  // dP = dO V^T
+                mma_kmajor<D>(tmem + C::COL_S + (g & 1) * TB, sbase + C::OFF_Q, sbase + C::k_slot(ks));
+                mma_commit(bar(C::BAR_SFULL + (g & 1)));
+                return true;
+            };
+            auto issue_dp = [&](int g) -> bool {
+                const int vs = g % C::NV;
+                if (!mbar_wait(bar(C::BAR_FULLV + vs), (g / C::NV) & 1, abort_flag, p.wait_limit_ns,
+                               p.status))
+                    return false;
+                tc_fence_after();
+                mma_kmajor<D>(tmem + C::COL_DP, sbase + C::OFF_DO, sbase + C::v_slot(vs));
                 mma_commit(bar(C::BAR_DPFULL));
-            }
+                mma_commit(bar(C::BAR_EMPTYV + vs));
+                return true;
+            };
+            bool ok = mbar_wait(bar(C::BAR_RES), 0, abort_flag, p.wait_limit_ns, p.status) && issue_s(0) &&
+                      issue_dp(0) && (n_kt < 2 || issue_s(1));
             for (int g = 0; ok && g < n_kt; ++g) {
-                const int st = g % C::NS, st1 = (g + 1) % C::NS;
-                const uint32_t k_s = sbase + C::stage(st), k_s1 = sbase + C::stage(st1);
-                if (g + 1 < n_kt) {
-                    if (!(ok = mbar_wait(bar(C::BAR_PDONE), g & 1, abort_flag, p.wait_limit_ns,
-                                         p.status)) ||
-                        !(ok = mbar_wait(bar(C::BAR_FULL + st1), ((g + 1) / C::NS) & 1, abort_flag,
-                                         p.wait_limit_ns, p.status)))
-                        break;
-                    tc_fence_after();
-                    mma_kmajor<D>(tmem + C::COL_S, sbase + C::OFF_R0, k_s1);
-                    mma_commit(bar(C::BAR_SFULL));
-                }
                 if (!(ok = mbar_wait(bar(C::BAR_DSFULL), g & 1, abort_flag, p.wait_limit_ns, p.status)))
                     break;
                 tc_fence_after();
-                mma_tmem_a<D, false>(tmem + C::COL_A, tmem + COL_DS, k_s, g > 0);  // dQ += dS K
-                mma_commit(bar(C::BAR_EMPTY + st));
-                if (g + 1 < n_kt) {
-                    mma_kmajor<D>(tmem + C::COL_DP, sbase + C::OFF_R1, k_s1 + C::TILE);
-                    mma_commit(bar(C::BAR_DPFULL));
-                }
+                mma_tmem_a<D, true>(tmem + C::COL_DQ, tmem + C::COL_S + (g & 1) * TB,
+                                    sbase + C::k_slot(g % C::NK), g > 0);  // dQ += dS K
+                mma_commit(bar(C::BAR_EMPTYK + g % C::NK));
+                if (g + 1 < n_kt && !(ok = issue_dp(g + 1))) break;
+                if (g + 2 < n_kt && !(ok = issue_s(g + 2))) break;
             }
             if (ok) mma_commit(bar(C::BAR_DONE));
         }
     } else {
-        // ===================== dS and the epilogue =====================
+        // ===================== P, dS and the epilogue =====================
         const int quad = warp & 3, half = warp >> 2;
         const int r = quad * 32 + lane;  // query row of the tile = TMEM lane
         const int i = q0 + r;
@@ -571,11 +617,13 @@ __global__ void __launch_bounds__(kThreadsTc, 1)
         const float del = i < p.Sq ? p.delta[qrow + i] : 0.f;
         bool ok = true;
         for (int g = 0; g < n_kt; ++g) {
-            if (!warp_wait(bar(C::BAR_SFULL), g & 1, abort_flag, p.wait_limit_ns, p.status)) {
+            if (!warp_wait(bar(C::BAR_SFULL + (g & 1)), (g >> 1) & 1, abort_flag, p.wait_limit_ns,
+                           p.status)) {
                 ok = false;
                 break;
             }
             tc_fence_after();
+            const uint32_t t_s = trow + C::COL_S + (g & 1) * TB + cb;
             const int kv0 = (lo + g) * TB;
             int clo, chi;
             cols_of_query(p, i, kv0, k_end, q_end, clo, chi);
@@ -584,8 +632,8 @@ __global__ void __launch_bounds__(kThreadsTc, 1)
             float pr[64];
             {
                 uint32_t sv[2][32];
-                tmem_ld32(trow + C::COL_S + cb, sv[0]);
-                tmem_ld32(trow + C::COL_S + cb + 32, sv[1]);
+                tmem_ld32(t_s, sv[0]);
+                tmem_ld32(t_s + 32, sv[1]);
                 tmem_wait_ld();
                 reg_fence32(sv[0]);
                 reg_fence32(sv[1]);
@@ -595,8 +643,6 @@ __global__ void __launch_bounds__(kThreadsTc, 1)
                     pr[x] = (x >= clo && x < chi) ? v : 0.f;
                 }
             }
-            tc_fence_before();
-            mbar_arrive(bar(C::BAR_PDONE));
             if (!warp_wait(bar(C::BAR_DPFULL), g & 1, abort_flag, p.wait_limit_ns, p.status)) {
                 ok = false;
                 break;
@@ -615,10 +661,10 @@ __global__ void __launch_bounds__(kThreadsTc, 1)
 #pragma unroll
                     for (int k = 0; k < 16; ++k) {
                         const int x = 32 * c + 2 * k;
-                        pk[k] = pack_bf16x2(pr[x] * (__uint_as_float(dv[x >> 5][x & 31]) - del),
-                                            pr[x + 1] * (__uint_as_float(dv[(x + 1) >> 5][(x + 1) & 31]) - del));
+                        pk[k] = pack_bf16x2(pr[x] * (__uint_as_float(dv[c][2 * k]) - del),
+                                            pr[x + 1] * (__uint_as_float(dv[c][2 * k + 1]) - del));
                     }
-                    tmem_st16(trow + C::COL_B + half * 32 + 16 * c, pk);
+                    tmem_st16(t_s + 16 * c, pk);  // dS over this warp's own S columns
                 }
             }
             tmem_wait_st();
@@ -629,12 +675,12 @@ __global__ void __launch_bounds__(kThreadsTc, 1)
                           warp_wait(bar(C::BAR_DONE), 0, abort_flag, p.wait_limit_ns, p.status);
         if (have) {
             tc_fence_after();
-            tc_store_half<D>(trow + C::COL_A, p.dQ + (qrow + i) * D, half * (D / 2), p.scale, i < p.Sq);
+            tc_store_half<D>(trow + C::COL_DQ, p.dQ + (qrow + i) * D, half * (D / 2), p.scale, i < p.Sq);
         } else if (i < p.Sq && !*abort_flag) {
             tc_zero_half<D>(p.dQ + (qrow + i) * D, half * (D / 2));
         }
     }
-    tc_teardown<D>(smem, tmem);
+    tc_teardown<C>(smem, tmem);
 }
 
 template <int D>
@@ -651,7 +697,7 @@ attn_status_t launch_bwd_tc_d(const BwdArgs &a, cudaStream_t stream) {
         if (cudaFuncSetAttribute(bwd_dkdv_tc_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                  C::SMEM) != cudaSuccess ||
             cudaFuncSetAttribute(bwd_dq_tc_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 C::SMEM) != cudaSuccess)
+                                 DqCfg<D>::SMEM) != cudaSuccess)
             return ATTN_ERR_CUDA;
         configured = true;
     }
@@ -678,14 +724,16 @@ attn_status_t launch_bwd_tc_d(const BwdArgs &a, cudaStream_t stream) {
     p.status = device_status_word();
     if (!p.status) return ATTN_ERR_CUDA;
     if (a.Sk > 0) {
-        bwd_dkdv_tc_kernel<D><<<dim3((a.Sk + TB - 1) / TB, a.Hkv, a.B), kThreadsTc, C::SMEM, stream>>>(
+        const long long grid_kv = (long long)((a.Sk + TB - 1) / TB) * a.Hkv * a.B;
+        if (grid_kv > 0x7fffffffll) return ATTN_ERR_INVALID;
+        bwd_dkdv_tc_kernel<D><<<static_cast<unsigned>(grid_kv), kThreadsTc, C::SMEM, stream>>>(
             tq, tk, tv, tdo, p);
         if (cudaGetLastError() != cudaSuccess) return ATTN_ERR_CUDA;
     }
     const int n_qt = (a.Sq + TB - 1) / TB;
     const long long grid = (long long)n_qt * a.Hq * a.B;
     if (grid > 0x7fffffffll) return ATTN_ERR_INVALID;
-    bwd_dq_tc_kernel<D><<<static_cast<unsigned>(grid), kThreadsTc, C::SMEM, stream>>>(tq, tk, tv, tdo, p,
+    bwd_dq_tc_kernel<D><<<static_cast<unsigned>(grid), kThreadsTc, DqCfg<D>::SMEM, stream>>>(tq, tk, tv, tdo, p,
                                                                                      n_qt);
     return cudaGetLastError() == cudaSuccess ? ATTN_OK : ATTN_ERR_CUDA;
 }
