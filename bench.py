@@ -492,7 +492,7 @@ def time_backward(step, steps, warmup, peak):
             "ms_per_launch": ms, "flops_per_launch": flops, "launches": steps,
             "roofline": {"bound": "tensor", "achieved": tf, "peak": peak, "unit": "TFLOP/s",
                          "frac": tf / peak,
-                         "kernel": "bwd_dkdv_kernel<128> + bwd_dq_kernel<128> + bwd_delta_kernel<128>"}}
+                         "kernel": "bwd_dkdv_tc_kernel<128> + bwd_dq_tc_kernel<128> + bwd_delta_kernel<128>"}}
 
 
 def time_paged(step, steps, warmup, peak):

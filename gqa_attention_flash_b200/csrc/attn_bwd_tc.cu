@@ -235,8 +235,9 @@ __global__ void __launch_bounds__(kThreadsTc, 1)
                        const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmdO,
                        const TcParams p) {
     using C = TcCfg<D>;
-    // key tiles in increasing order, the (KV head, batch) pairs fastest: under a
-    // causal mask the heaviest tiles go first
+    // (KV head, batch) pairs in chunks of 4; inside a chunk the key tiles in
+    // increasing order with the pairs fastest: under a causal mask the heaviest
+    // tiles go first, and the Q / dO rows one wave reads (a few chunks) stay in L2
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>(
         (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -244,8 +245,13 @@ __global__ void __launch_bounds__(kThreadsTc, 1)
     auto bar = [&](int i) -> uint32_t { return sbase + C::OFF_BAR + 8 * i; };
     volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + C::OFF_MISC + 4);
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int hkv = blockIdx.x % p.Hkv, b = (blockIdx.x / p.Hkv) % p.B,
-              kt = blockIdx.x / (p.Hkv * p.B);
+    const int pairs = p.Hkv * p.B, n_kt = (p.Sk + TB - 1) / TB;
+    const int G = min(4, pairs), full = pairs / G;
+    const int chunk = min(static_cast<int>(blockIdx.x / (G * n_kt)), full);
+    const int size = chunk < full ? G : pairs - full * G;
+    const int local = static_cast<int>(blockIdx.x) - chunk * G * n_kt;
+    const int kt = local / size, pair = chunk * G + local % size;
+    const int hkv = pair % p.Hkv, b = pair / p.Hkv;
     const int kv0 = kt * TB;
     int k_end, q_end;
     tc_lengths(p, b, k_end, q_end);
