@@ -52,6 +52,11 @@ CASES = [
     (2, 2, 1, 100, 300, 64, True, 0, 200, False),
     (1, 8, 2, 260, 260, 128, True, 70, 0, False),
     (3, 4, 2, 190, 190, 128, True, 0, 0, True),
+    # long enough that the dQ kernel's 3-slot K ring and 2-slot V ring and the dK/dV
+    # kernel's 2-slot Q/dO ring wrap several times
+    (1, 4, 2, 640, 640, 64, True, 0, 0, False),
+    (1, 2, 1, 300, 777, 128, False, 0, 0, False),
+    (2, 4, 1, 520, 520, 128, True, 200, 0, True),
 ]
 
 
