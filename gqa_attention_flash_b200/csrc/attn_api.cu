@@ -1,6 +1,6 @@
 // attn_api.cu -- the library's C ABI (declared in include/gqa_attn.h):
 // host-side argument validation, TMA descriptor encoding, the per-device status
-// word, and the decode workspace.
+// word, and the workspaces (from a per-device pool the library owns).
 #include <cmath>
 #include <cstdint>
 #include <cstring>
@@ -34,6 +34,43 @@ int *device_status_word() {
 }
 
 size_t decode_workspace_floats(int B, int Hq, int n_splits, int D);
+
+namespace {
+std::mutex g_pool_mutex;
+cudaMemPool_t g_pool[64] = {};
+bool g_pool_made[64] = {};
+}  // namespace
+
+// Stream-ordered workspace from a memory pool the library owns on each device
+// (made on first use).  Its release threshold is the maximum, so memory freed
+// back to it stays reserved for the next call instead of returning to the driver
+// at every synchronisation; the default pool, which other code in the process may
+// use, keeps its own settings.
+cudaError_t workspace_alloc(void **ptr, size_t bytes, cudaStream_t stream) {
+    int dev = -1;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
+    cudaMemPool_t pool;
+    {
+        std::lock_guard<std::mutex> lock(g_pool_mutex);
+        if (!g_pool_made[dev]) {
+            cudaMemPoolProps props = {};
+            props.allocType = cudaMemAllocationTypePinned;
+            props.handleTypes = cudaMemHandleTypeNone;
+            props.location.type = cudaMemLocationTypeDevice;
+            props.location.id = dev;
+            if ((e = cudaMemPoolCreate(&g_pool[dev], &props)) != cudaSuccess) return e;
+            uint64_t keep = UINT64_MAX;
+            if ((e = cudaMemPoolSetAttribute(g_pool[dev], cudaMemPoolAttrReleaseThreshold, &keep)) !=
+                cudaSuccess)
+                return e;
+            g_pool_made[dev] = true;
+        }
+        pool = g_pool[dev];
+    }
+    return cudaMallocFromPoolAsync(ptr, bytes, pool, stream);
+}
 
 namespace {
 
@@ -259,7 +296,7 @@ attn_status_t attn_decode(void *O, const void *Q, const void *K, const void *V,
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     const size_t bytes = decode_workspace_floats(B, Hq, n_splits, D) * sizeof(float);
     void *ws = nullptr;
-    if (cudaMallocAsync(&ws, bytes, s) != cudaSuccess) return ATTN_ERR_CUDA;
+    if (workspace_alloc(&ws, bytes, s) != cudaSuccess) return ATTN_ERR_CUDA;
     DecodeArgs a;
     a.O = O;
     a.Q = Q;
@@ -303,7 +340,7 @@ attn_status_t attn_bwd(void *dQ, void *dK, void *dV, const void *dO, const void 
         return ATTN_OK;
     }
     void *ws = nullptr;
-    if (cudaMallocAsync(&ws, (size_t)rows_q * sizeof(float), s) != cudaSuccess) return ATTN_ERR_CUDA;
+    if (workspace_alloc(&ws, (size_t)rows_q * sizeof(float), s) != cudaSuccess) return ATTN_ERR_CUDA;
     BwdArgs a;
     a.dQ = dQ;
     a.dK = dK;
@@ -352,7 +389,7 @@ attn_status_t attn_rbs_block_mask(uint8_t *block_mask, float *base_scores, float
     const size_t ws_floats = (size_t)B * Hkv * nkb * (D + 2);
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     void *ws = nullptr;
-    if (cudaMallocAsync(&ws, ws_floats * sizeof(float), s) != cudaSuccess) return ATTN_ERR_CUDA;
+    if (workspace_alloc(&ws, ws_floats * sizeof(float), s) != cudaSuccess) return ATTN_ERR_CUDA;
     RbsArgs a;
     a.Q = Q;
     a.K = K;
@@ -399,7 +436,7 @@ attn_status_t attn_decode_paged(void *O, const void *Q, const void *K_cache, con
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     const size_t bytes = decode_workspace_floats(B, Hq, n_splits, D) * sizeof(float);
     void *ws = nullptr;
-    if (cudaMallocAsync(&ws, bytes, s) != cudaSuccess) return ATTN_ERR_CUDA;
+    if (workspace_alloc(&ws, bytes, s) != cudaSuccess) return ATTN_ERR_CUDA;
     DecodeArgs a;
     a.O = O;
     a.Q = Q;

@@ -1,6 +1,6 @@
 // attn_decode_noalloc.cu -- split-KV decode for callers that must not allocate.
 //
-// attn_decode() obtains its per-slice workspace with cudaMallocAsync on every
+// attn_decode() obtains its per-slice workspace from a stream-ordered allocator on every
 // call.  Some callers cannot allow that: a serving loop that reserves all of its
 // device memory up front and forbids any allocation afterwards (an allocation
 // can fail once the memory is spoken for, and its latency is not bounded), or a

@@ -230,7 +230,8 @@ attn_status_t attn_block_mask_document(uint8_t *out, int Sq, int Sk, int input_p
  *
  * The per-slice partial results live in a workspace of
  * B * Hq * n_splits * (D + 4) floats that the call allocates and frees in
- * stream order (cudaMallocAsync / cudaFreeAsync on `stream`).
+ * stream order on `stream`, from a memory pool the library keeps per device
+ * (memory freed to it stays reserved for later calls).
  */
 attn_status_t attn_decode(void *O, const void *Q, const void *K, const void *V,
                           const int32_t *lengths, int n_splits, void *stream,
@@ -265,8 +266,8 @@ attn_status_t attn_decode_paged(void *O, const void *Q, const void *K_cache, con
  * memory.  The pages have no counterpart: it is attn_decode with a different
  * home for the per-slice workspace.
  *
- * Who needs it: attn_decode calls cudaMallocAsync / cudaFreeAsync on every
- * call.  A serving loop that reserves all of its device memory up front and
+ * Who needs it: attn_decode allocates and frees its workspace (stream
+ * ordered, from the library's pool) on every call.  A serving loop that reserves all of its device memory up front and
  * forbids allocation afterwards (an allocation can fail once the memory is
  * spoken for, and its latency is not bounded), or a program whose device
  * memory belongs to another allocator, cannot let the library allocate.  This
