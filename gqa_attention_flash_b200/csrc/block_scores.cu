@@ -16,12 +16,19 @@
 //                        (<q, c> + |q| r beta) / sqrt(D) for the block's query
 //                        tokens, log-sum-exp over the tokens, then the row's
 //                        relative mask: keep where score >= row max + ln alpha in
-//                        either branch, or |qb - kb| < diagonal.
+//                        either branch, or |qb - kb| < diagonal.  <q, c> for the
+//                        64 tokens and 64 key blocks at a time is a 64 x 64 x D
+//                        product on the tensor cores (warp-level bf16 MMA, fp32
+//                        accumulation) with each centroid split into a bf16 high
+//                        part and a bf16 remainder, so the two products together
+//                        carry the fp32 centroid to ~2^-17 relative (the queries
+//                        are bf16 already).
 // The mask is written as BlockMask states (2 = keep the whole block, 0 = skip),
 // one (nqb, nkb) matrix per (batch, query head), ready for attn_fwd_flex.
 #include <cuda_bf16.h>
 
 #include "internal.h"
+#include "sm100_ptx.cuh"
 
 namespace gqa {
 
@@ -31,8 +38,9 @@ constexpr int kBlk = 64;
 
 template <int D>
 __global__ void __launch_bounds__(128)
-    rbs_centroid_kernel(const __nv_bfloat16 *__restrict__ K, float *__restrict__ cent,
-                        float *__restrict__ rad, int Hkv, int Sk, int nkb) {
+    rbs_centroid_kernel(const __nv_bfloat16 *__restrict__ K, __nv_bfloat16 *__restrict__ cent_hi,
+                        __nv_bfloat16 *__restrict__ cent_lo, float *__restrict__ rad, int Hkv, int Sk,
+                        int nkb) {
     __shared__ __align__(16) __nv_bfloat16 kblk[kBlk * D];  // the key block, read once
     __shared__ float c[D];
     __shared__ float rmax_w[4];
@@ -63,7 +71,11 @@ __global__ void __launch_bounds__(128)
     }
     if (lane == 0) rmax_w[warp] = rm;
     const long long row = (long long)(b * Hkv + hkv) * nkb + kb;
-    if (tid < D) cent[row * D + tid] = c[tid];
+    if (tid < D) {  // the centroid as bf16 high part + bf16 remainder
+        const __nv_bfloat16 hi = __float2bfloat16_rn(c[tid]);
+        cent_hi[row * D + tid] = hi;
+        cent_lo[row * D + tid] = __float2bfloat16_rn(c[tid] - __bfloat162float(hi));
+    }
     __syncthreads();
     if (tid == 0) rad[row] = fmaxf(fmaxf(rmax_w[0], rmax_w[1]), fmaxf(rmax_w[2], rmax_w[3]));
 }
@@ -112,7 +124,8 @@ __global__ void __launch_bounds__(256)
 
 struct ScoreParams {
     const __nv_bfloat16 *Q;
-    const float *cent, *rad, *beta;
+    const __nv_bfloat16 *cent_hi, *cent_lo;
+    const float *rad, *beta;
     uint8_t *mask;
     float *base_out, *rescue_out;  // optional
     int Hq, Hkv, group, Sq, nqb, nkb;
@@ -120,85 +133,147 @@ struct ScoreParams {
     int diagonal;
 };
 
+// Byte offset of 16-byte chunk c of row `row` in a 64-row bf16 tile stored as
+// D/64 boxes of (64 rows x 128 bytes) with the 128-byte XOR swizzle, so that
+// ldmatrix reads of 8 rows at one chunk hit 8 different bank groups.
+__device__ __forceinline__ uint32_t swz64(int row, int c) {
+    return static_cast<uint32_t>((c >> 3) * (64 * 128) + row * 128 + (((c & 7) ^ (row & 7)) << 4));
+}
+
+// Rows [0, n) of a row-major (., D) bf16 matrix into a swizzled 64-row tile
+// (rows n..63 zero), 16-byte loads spread over the block's threads.
 template <int D>
-__global__ void __launch_bounds__(256) rbs_scores_kernel(const ScoreParams p) {
-    extern __shared__ float sm[];
-    constexpr int kLd = kBlk + 1;         // padded row: conflict-free transposed stores
-    float *qT = sm;                       // [D][kLd] query block, transposed
-    constexpr int kCg = 64;               // key blocks per group (8 per warp)
-    constexpr int kCld = kCg + 4;         // padded row of the transposed centroids
-    float *qn = qT + D * kLd;             // [64] |q_t|
-    float *cT = qn + kBlk;                // [D][kCld] centroids of one group, transposed
-    float *sb = cT + D * kCld;            // [nkb] base scores of this row
+__device__ __forceinline__ void stage64(uint8_t *tile, const __nv_bfloat16 *src, int n) {
+    constexpr int kChunks = D / 8;
+    for (int i = threadIdx.x; i < 64 * kChunks; i += blockDim.x) {
+        const int row = i / kChunks, c = i % kChunks;
+        uint4 v = make_uint4(0, 0, 0, 0);
+        if (row < n) v = __ldg(reinterpret_cast<const uint4 *>(src + (long long)row * D) + c);
+        *reinterpret_cast<uint4 *>(tile + swz64(row, c)) = v;
+    }
+}
+
+template <int D>
+__global__ void __launch_bounds__(128) rbs_scores_kernel(const ScoreParams p) {
+    extern __shared__ __align__(1024) uint8_t smraw[];
+    constexpr int kKs = D / 16;           // k-steps of 16
+    constexpr int kTile = 64 * D * 2;     // bytes of one staged 64-row tile
+    uint8_t *q_tile = smraw;              // the query block
+    uint8_t *ch_tile = smraw + kTile;     // centroids of a 64-block group: high parts
+    uint8_t *cl_tile = smraw + 2 * kTile; // ... remainders
+    float *red = reinterpret_cast<float *>(smraw + 3 * kTile);  // [4][64][2 branches][max, sum]
+    float *sb = red + 4 * 64 * 4;         // [nkb] base scores of this row
     float *sr = sb + p.nkb;               // [nkb] rescue scores
-    __shared__ float red[2][8];
+    __shared__ float red2[2][4];
     const int qb = blockIdx.x, hq = blockIdx.y, b = blockIdx.z;
     const int hkv = hq / p.group;
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int g = lane >> 2, t = lane & 3;
+    const int mi = lane >> 3, rr = lane & 7;  // ldmatrix: matrix of this lane's address, its row
     const int i0 = qb * kBlk, n_rows = min(kBlk, p.Sq - i0);
-    const __nv_bfloat16 *Qb = p.Q + ((long long)(b * p.Hq + hq) * p.Sq + i0) * D;
-    for (int idx = tid; idx < kBlk * D; idx += blockDim.x) {
-        const int t = idx / D, d = idx % D;
-        qT[d * kLd + t] = t < n_rows ? __bfloat162float(Qb[(long long)t * D + d]) : 0.f;
-    }
-    __syncthreads();
-    if (tid < kBlk) {
-        float ss = 0.f;
-        for (int d = 0; d < D; ++d) ss = fmaf(qT[d * kLd + tid], qT[d * kLd + tid], ss);
-        qn[tid] = sqrtf(ss);
-    }
-    __syncthreads();
-    const float inv_sqrt_d = rsqrtf(static_cast<float>(D));
     const long long hrow = (long long)(b * p.Hkv + hkv) * p.nkb;
-    const bool v0 = lane < n_rows, v1 = lane + 32 < n_rows;
+    stage64<D>(q_tile, p.Q + ((long long)(b * p.Hq + hq) * p.Sq + i0) * D, n_rows);
+    // this warp's 16 token rows as m16n8k16 A fragments (rows r and r + 8)
+    const int r = warp * 16 + g;
+    const bool v0 = r < n_rows, v1 = r + 8 < n_rows;
+    const float inv_sqrt_d = rsqrtf(static_cast<float>(D));
     const float ninf = __int_as_float(0xff800000);
-    // Key blocks in groups of 64: the group's centroids are staged transposed in
-    // shared memory; warp w takes 8 of them and each lane 2 query rows, so every
-    // shared-memory read feeds 4 or 16 FMAs (register blocking).
-    for (int g0 = 0; g0 < p.nkb; g0 += kCg) {
-        for (int idx = tid; idx < kCg * D; idx += blockDim.x) {
-            const int j = idx / D, d = idx % D;
-            cT[d * kCld + j] = g0 + j < p.nkb ? p.cent[(hrow + g0 + j) * D + d] : 0.f;
-        }
+    const uint32_t qs = smem_u32(q_tile), hs = smem_u32(ch_tile), ls = smem_u32(cl_tile);
+    uint32_t a[kKs][4];
+    float qn0 = 0.f, qn1 = 0.f;
+    // key blocks in groups of 64 = 8 n-tiles of 8
+    for (int g0 = 0; g0 < p.nkb; g0 += 64) {
+        const int nk = min(64, p.nkb - g0);
+        stage64<D>(ch_tile, p.cent_hi + (hrow + g0) * D, nk);
+        stage64<D>(cl_tile, p.cent_lo + (hrow + g0) * D, nk);
         __syncthreads();
-        float acc0[8], acc1[8];
+        if (g0 == 0) {
+            float q0 = 0.f, q1 = 0.f;  // partial |q|^2 of rows r, r + 8
 #pragma unroll
-        for (int j = 0; j < 8; ++j) acc0[j] = acc1[j] = 0.f;
-#pragma unroll 4
-        for (int d = 0; d < D; ++d) {
-            const float q0 = qT[d * kLd + lane], q1 = qT[d * kLd + lane + 32];
-            const float4 ca = *reinterpret_cast<const float4 *>(cT + d * kCld + 8 * warp);
-            const float4 cb = *reinterpret_cast<const float4 *>(cT + d * kCld + 8 * warp + 4);
-            const float cv[8] = {ca.x, ca.y, ca.z, ca.w, cb.x, cb.y, cb.z, cb.w};
+            for (int kk = 0; kk < kKs; ++kk) {
+                ldmatrix_x4(qs + swz64(warp * 16 + (mi & 1) * 8 + rr, 2 * kk + (mi >> 1)), a[kk][0],
+                            a[kk][1], a[kk][2], a[kk][3]);
 #pragma unroll
-            for (int j = 0; j < 8; ++j) {
-                acc0[j] = fmaf(q0, cv[j], acc0[j]);
-                acc1[j] = fmaf(q1, cv[j], acc1[j]);
+                for (int e = 0; e < 4; ++e) {
+                    const __nv_bfloat162 h = *reinterpret_cast<const __nv_bfloat162 *>(&a[kk][e]);
+                    const float x = __low2float(h), y = __high2float(h);
+                    if (e & 1) q1 = fmaf(x, x, fmaf(y, y, q1));
+                    else q0 = fmaf(x, x, fmaf(y, y, q0));
+                }
+            }
+            q0 += __shfl_xor_sync(0xffffffffu, q0, 1);
+            q0 += __shfl_xor_sync(0xffffffffu, q0, 2);
+            q1 += __shfl_xor_sync(0xffffffffu, q1, 1);
+            q1 += __shfl_xor_sync(0xffffffffu, q1, 2);
+            qn0 = sqrtf(q0);
+            qn1 = sqrtf(q1);
+        }
+        float acc[8][4];
+#pragma unroll
+        for (int j = 0; j < 8; ++j) acc[j][0] = acc[j][1] = acc[j][2] = acc[j][3] = 0.f;
+#pragma unroll
+        for (int kk = 0; kk < kKs; ++kk) {
+#pragma unroll
+            for (int jp = 0; jp < 4; ++jp) {  // n-tiles 2 jp, 2 jp + 1
+                const uint32_t off = swz64(16 * jp + (mi >> 1) * 8 + rr, 2 * kk + (mi & 1));
+                uint32_t h0, h1, h2, h3, l0, l1, l2, l3;
+                ldmatrix_x4(hs + off, h0, h1, h2, h3);
+                ldmatrix_x4(ls + off, l0, l1, l2, l3);
+                mma_m16n8k16(acc[2 * jp], a[kk], h0, h1);
+                mma_m16n8k16(acc[2 * jp], a[kk], l0, l1);
+                mma_m16n8k16(acc[2 * jp + 1], a[kk], h2, h3);
+                mma_m16n8k16(acc[2 * jp + 1], a[kk], l2, l3);
             }
         }
+        // per key block: log-sum-exp of each branch over this warp's 16 rows
 #pragma unroll
         for (int j = 0; j < 8; ++j) {
-            const int kb = g0 + 8 * warp + j;
-            if (kb >= p.nkb) break;  // warp-uniform
-            const float rb = p.rad[hrow + kb] * p.beta[hrow + kb];
-            const float b0 = v0 ? acc0[j] * inv_sqrt_d : ninf, b1 = v1 ? acc1[j] * inv_sqrt_d : ninf;
-            const float r0 = v0 ? fmaf(qn[lane], rb, acc0[j]) * inv_sqrt_d : ninf;
-            const float r1 = v1 ? fmaf(qn[lane + 32], rb, acc1[j]) * inv_sqrt_d : ninf;
-            float mb = fmaxf(b0, b1), mr = fmaxf(r0, r1);
 #pragma unroll
-            for (int o = 16; o > 0; o >>= 1) {
-                mb = fmaxf(mb, __shfl_xor_sync(0xffffffffu, mb, o));
-                mr = fmaxf(mr, __shfl_xor_sync(0xffffffffu, mr, o));
-            }
-            float eb = __expf(b0 - mb) + __expf(b1 - mb), er = __expf(r0 - mr) + __expf(r1 - mr);
+            for (int e = 0; e < 2; ++e) {
+                const int col = 8 * j + 2 * t + e;  // key block g0 + col
+                const int kb = g0 + col;
+                const float rb = kb < p.nkb ? p.rad[hrow + kb] * p.beta[hrow + kb] : 0.f;
+                const float s0 = acc[j][e], s1 = acc[j][2 + e];
+                const float b0 = v0 ? s0 * inv_sqrt_d : ninf, b1 = v1 ? s1 * inv_sqrt_d : ninf;
+                const float x0 = v0 ? fmaf(qn0, rb, s0) * inv_sqrt_d : ninf;
+                const float x1 = v1 ? fmaf(qn1, rb, s1) * inv_sqrt_d : ninf;
+                float mb = fmaxf(b0, b1), mr = fmaxf(x0, x1);
 #pragma unroll
-            for (int o = 16; o > 0; o >>= 1) {
-                eb += __shfl_xor_sync(0xffffffffu, eb, o);
-                er += __shfl_xor_sync(0xffffffffu, er, o);
+                for (int o = 4; o < 32; o <<= 1) {
+                    mb = fmaxf(mb, __shfl_xor_sync(0xffffffffu, mb, o));
+                    mr = fmaxf(mr, __shfl_xor_sync(0xffffffffu, mr, o));
+                }
+                // a warp with no valid row has m = -inf: contribute (m, 0)
+                float eb = mb == ninf ? 0.f : __expf(b0 - mb) + __expf(b1 - mb);
+                float er = mr == ninf ? 0.f : __expf(x0 - mr) + __expf(x1 - mr);
+#pragma unroll
+                for (int o = 4; o < 32; o <<= 1) {
+                    eb += __shfl_xor_sync(0xffffffffu, eb, o);
+                    er += __shfl_xor_sync(0xffffffffu, er, o);
+                }
+                if (g == 0) {
+                    float *w = red + ((warp * 64 + col) * 2) * 2;
+                    w[0] = mb;
+                    w[1] = eb;
+                    w[2] = mr;
+                    w[3] = er;
+                }
             }
-            if (lane == 0) {
-                sb[kb] = mb + __logf(eb);
-                sr[kb] = mr + __logf(er);
+        }
+        __syncthreads();
+        if (tid < 64 && g0 + tid < p.nkb) {  // combine the four warps
+#pragma unroll
+            for (int br = 0; br < 2; ++br) {
+                float m = ninf;
+#pragma unroll
+                for (int w = 0; w < 4; ++w) m = fmaxf(m, red[((w * 64 + tid) * 2 + br) * 2]);
+                float sum = 0.f;
+#pragma unroll
+                for (int w = 0; w < 4; ++w) {
+                    const float mw = red[((w * 64 + tid) * 2 + br) * 2];
+                    if (mw != ninf) sum += red[((w * 64 + tid) * 2 + br) * 2 + 1] * __expf(mw - m);
+                }
+                (br ? sr : sb)[g0 + tid] = m + __logf(sum);
             }
         }
         __syncthreads();
@@ -216,16 +291,16 @@ __global__ void __launch_bounds__(256) rbs_scores_kernel(const ScoreParams p) {
         mr = fmaxf(mr, __shfl_xor_sync(0xffffffffu, mr, o));
     }
     if (lane == 0) {
-        red[0][warp] = mb;
-        red[1][warp] = mr;
+        red2[0][warp] = mb;
+        red2[1][warp] = mr;
     }
     __syncthreads();
-    mb = red[0][0];
-    mr = red[1][0];
+    mb = red2[0][0];
+    mr = red2[1][0];
 #pragma unroll
-    for (int w = 1; w < 8; ++w) {
-        mb = fmaxf(mb, red[0][w]);
-        mr = fmaxf(mr, red[1][w]);
+    for (int w = 1; w < 4; ++w) {
+        mb = fmaxf(mb, red2[0][w]);
+        mr = fmaxf(mr, red2[1][w]);
     }
     const long long orow = ((long long)(b * p.Hq + hq) * p.nqb + qb) * p.nkb;
     for (int kb = tid; kb < p.nkb; kb += blockDim.x) {
@@ -240,8 +315,11 @@ __global__ void __launch_bounds__(256) rbs_scores_kernel(const ScoreParams p) {
 template <int D>
 attn_status_t launch_rbs_d(const RbsArgs &a, cudaStream_t stream) {
     const int nqb = (a.Sq + kBlk - 1) / kBlk, nkb = (a.Sk + kBlk - 1) / kBlk;
+    // the fp32 centroid workspace holds the bf16 high parts and then the remainders
+    __nv_bfloat16 *cent_hi = reinterpret_cast<__nv_bfloat16 *>(a.cent);
+    __nv_bfloat16 *cent_lo = cent_hi + (size_t)a.B * a.Hkv * nkb * D;
     rbs_centroid_kernel<D><<<dim3(nkb, a.Hkv, a.B), 128, 0, stream>>>(
-        static_cast<const __nv_bfloat16 *>(a.K), a.cent, a.rad, a.Hkv, a.Sk, nkb);
+        static_cast<const __nv_bfloat16 *>(a.K), cent_hi, cent_lo, a.rad, a.Hkv, a.Sk, nkb);
     if (cudaGetLastError() != cudaSuccess) return ATTN_ERR_CUDA;
     int n_pow2 = 1;
     while (n_pow2 < nkb) n_pow2 <<= 1;
@@ -250,7 +328,8 @@ attn_status_t launch_rbs_d(const RbsArgs &a, cudaStream_t stream) {
     if (cudaGetLastError() != cudaSuccess) return ATTN_ERR_CUDA;
     ScoreParams p;
     p.Q = static_cast<const __nv_bfloat16 *>(a.Q);
-    p.cent = a.cent;
+    p.cent_hi = cent_hi;
+    p.cent_lo = cent_lo;
     p.rad = a.rad;
     p.beta = a.beta;
     p.mask = a.mask;
@@ -265,8 +344,7 @@ attn_status_t launch_rbs_d(const RbsArgs &a, cudaStream_t stream) {
     p.ln_alpha_base = logf(a.alpha_base);
     p.ln_alpha_rescue = logf(a.alpha_rescue);
     p.diagonal = a.diagonal;
-    const size_t smem = sizeof(float) * ((size_t)D * (kBlk + 1) + kBlk + (size_t)D * (64 + 4) +
-                                         2 * (size_t)nkb);
+    const size_t smem = 3 * (size_t)64 * D * 2 + sizeof(float) * (4 * 64 * 4 + 2 * (size_t)nkb);
     static bool configured = false;
     if (!configured) {
         if (cudaFuncSetAttribute(rbs_scores_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -274,7 +352,7 @@ attn_status_t launch_rbs_d(const RbsArgs &a, cudaStream_t stream) {
             return ATTN_ERR_CUDA;
         configured = true;
     }
-    rbs_scores_kernel<D><<<dim3(nqb, a.Hq, a.B), 256, smem, stream>>>(p);
+    rbs_scores_kernel<D><<<dim3(nqb, a.Hq, a.B), 128, smem, stream>>>(p);
     return cudaGetLastError() == cudaSuccess ? ATTN_OK : ATTN_ERR_CUDA;
 }
 
