@@ -5,6 +5,8 @@
 #include <cstdint>
 #include <cstring>
 #include <mutex>
+#include <set>
+#include <utility>
 
 #include <cuda.h>
 #include <cuda_runtime.h>
@@ -34,6 +36,29 @@ int *device_status_word() {
 }
 
 size_t decode_workspace_floats(int B, int Hq, int n_splits, int D);
+
+namespace {
+std::mutex g_setup_mutex;
+std::set<std::pair<int, const void *>> g_setup_done;
+}  // namespace
+
+cudaError_t kernel_setup(const void *func, int smem_bytes, int required_regs) {
+    int dev = -1;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    std::lock_guard<std::mutex> lock(g_setup_mutex);
+    if (g_setup_done.count({dev, func})) return cudaSuccess;
+    if (required_regs >= 0) {
+        cudaFuncAttributes fa;
+        if ((e = cudaFuncGetAttributes(&fa, func)) != cudaSuccess) return e;
+        if (fa.numRegs != required_regs) return cudaErrorInvalidValue;
+    }
+    if ((e = cudaFuncSetAttribute(func, cudaFuncAttributeMaxDynamicSharedMemorySize, smem_bytes)) !=
+        cudaSuccess)
+        return e;
+    g_setup_done.insert({dev, func});
+    return cudaSuccess;
+}
 
 namespace {
 std::mutex g_pool_mutex;

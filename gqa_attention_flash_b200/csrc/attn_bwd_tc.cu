@@ -698,15 +698,10 @@ attn_status_t launch_bwd_tc_d(const BwdArgs &a, cudaStream_t stream) {
     if ((st = make_tmap_bf16_3d(&tdo, a.dO, D, a.Sq, (uint64_t)a.B * a.Hq, TB)) != ATTN_OK) return st;
     if ((st = make_tmap_bf16_3d(&tk, a.K, D, a.Sk, (uint64_t)a.B * a.Hkv, TB)) != ATTN_OK) return st;
     if ((st = make_tmap_bf16_3d(&tv, a.V, D, a.Sk, (uint64_t)a.B * a.Hkv, TB)) != ATTN_OK) return st;
-    static bool configured = false;
-    if (!configured) {
-        if (cudaFuncSetAttribute(bwd_dkdv_tc_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 C::SMEM) != cudaSuccess ||
-            cudaFuncSetAttribute(bwd_dq_tc_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 DqCfg<D>::SMEM) != cudaSuccess)
-            return ATTN_ERR_CUDA;
-        configured = true;
-    }
+    if (kernel_setup(reinterpret_cast<const void *>(bwd_dkdv_tc_kernel<D>), C::SMEM) != cudaSuccess ||
+        kernel_setup(reinterpret_cast<const void *>(bwd_dq_tc_kernel<D>), DqCfg<D>::SMEM) !=
+            cudaSuccess)
+        return ATTN_ERR_CUDA;
     TcParams p;
     p.LSE = a.LSE;
     p.delta = a.delta;

@@ -404,14 +404,9 @@ attn_status_t launch_decode_d(const DecodeArgs &a, cudaStream_t stream) {
         if ((st = make_tmap_bf16_3d(&tv, a.V, D, a.S_cap, (uint64_t)a.B * a.Hkv, TN)) != ATTN_OK)
             return st;
     }
-    static bool configured = false;
-    if (!configured) {
-        if (cudaFuncSetAttribute(decode_split_kernel<D, kPaged>,
-                                 cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 C::SMEM_BYTES) != cudaSuccess)
-            return ATTN_ERR_CUDA;
-        configured = true;
-    }
+    if (kernel_setup(reinterpret_cast<const void *>(decode_split_kernel<D, kPaged>), C::SMEM_BYTES) !=
+        cudaSuccess)
+        return ATTN_ERR_CUDA;
     DecParams p;
     p.Q = static_cast<const __nv_bfloat16 *>(a.Q);
     p.ws = a.workspace;

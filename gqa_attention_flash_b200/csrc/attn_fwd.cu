@@ -704,19 +704,11 @@ attn_status_t launch_fwd_d(const FwdArgs &a, cudaStream_t stream) {
     if ((st = make_tmap_bf16_3d(&tq, a.Q, D, a.Sq, (uint64_t)a.B * a.Hq, BM)) != ATTN_OK) return st;
     if ((st = make_tmap_bf16_3d(&tk, a.K, D, a.Sk, (uint64_t)a.B * a.Hkv, BN)) != ATTN_OK) return st;
     if ((st = make_tmap_bf16_3d(&tv, a.V, D, a.Sk, (uint64_t)a.B * a.Hkv, BN)) != ATTN_OK) return st;
-    static bool configured = false;
-    if (!configured) {
-        // The register hand-over inside the kernel assumes exactly kLaunchRegs
-        // registers per thread at launch; refuse to launch a build where it differs.
-        cudaFuncAttributes fa;
-        if (cudaFuncGetAttributes(&fa, attn_fwd_kernel<D, kMode, kList>) != cudaSuccess ||
-            fa.numRegs != kLaunchRegs)
-            return ATTN_ERR_CUDA;
-        if (cudaFuncSetAttribute(attn_fwd_kernel<D, kMode, kList>,
-                                 cudaFuncAttributeMaxDynamicSharedMemorySize, kSmem) != cudaSuccess)
-            return ATTN_ERR_CUDA;
-        configured = true;
-    }
+    // The register hand-over inside the kernel assumes exactly kLaunchRegs
+    // registers per thread at launch; refuse to launch a build where it differs.
+    if (kernel_setup(reinterpret_cast<const void *>(attn_fwd_kernel<D, kMode, kList>), kSmem,
+                     kLaunchRegs) != cudaSuccess)
+        return ATTN_ERR_CUDA;
     FwdParams p;
     p.O = static_cast<__nv_bfloat16 *>(a.O);
     p.LSE = a.LSE;

@@ -345,13 +345,8 @@ attn_status_t launch_rbs_d(const RbsArgs &a, cudaStream_t stream) {
     p.ln_alpha_rescue = logf(a.alpha_rescue);
     p.diagonal = a.diagonal;
     const size_t smem = 3 * (size_t)64 * D * 2 + sizeof(float) * (4 * 64 * 4 + 2 * (size_t)nkb);
-    static bool configured = false;
-    if (!configured) {
-        if (cudaFuncSetAttribute(rbs_scores_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 100 * 1024) != cudaSuccess)
-            return ATTN_ERR_CUDA;
-        configured = true;
-    }
+    if (kernel_setup(reinterpret_cast<const void *>(rbs_scores_kernel<D>), 100 * 1024) != cudaSuccess)
+        return ATTN_ERR_CUDA;
     rbs_scores_kernel<D><<<dim3(nqb, a.Hq, a.B), 128, smem, stream>>>(p);
     return cudaGetLastError() == cudaSuccess ? ATTN_OK : ATTN_ERR_CUDA;
 }

@@ -91,6 +91,11 @@ attn_status_t launch_fwd(const FwdArgs &a, cudaStream_t stream);
 attn_status_t launch_decode(const DecodeArgs &a, cudaStream_t stream);
 attn_status_t launch_wait_probe(int limit_us, cudaStream_t stream);
 
+// Once per (device, kernel), thread-safe: check that the kernel was built with
+// `required_regs` registers per thread (skipped when negative) and raise its
+// dynamic shared-memory limit to `smem_bytes` on the current device.
+cudaError_t kernel_setup(const void *func, int smem_bytes, int required_regs = -1);
+
 // Bounded-wait limit used by the attention kernels (nanoseconds of global time).
 constexpr uint64_t kWaitLimitNs = 2000000000ull;
 
