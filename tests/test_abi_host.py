@@ -219,3 +219,26 @@ def test_rbs_host_validation(binding):
     assert rbs(mask=None) == 1
     assert rbs(Q=ctypes.c_void_p(20)) == 2
     assert rbs(B=0) == 0
+
+
+def test_bwd_host_validation(binding):
+    L = binding.lib
+
+    def bwd(**kw):
+        a = dict(dQ=P, dK=P, dV=P, dO=P, Q=P, K=P, V=P, O=P, LSE=P, B=1, Hq=2, Hkv=1, Sq=4, Sk=4,
+                 D=128, scale=0.1, causal=1, window=0, input_pos=0)
+        a.update(kw)
+        return L.attn_bwd(a["dQ"], a["dK"], a["dV"], a["dO"], a["Q"], a["K"], a["V"], a["O"],
+                          a["LSE"], a["B"], a["Hq"], a["Hkv"], a["Sq"], a["Sk"], a["D"], a["scale"],
+                          a["causal"], a["window"], a["input_pos"], None, None, None)
+    assert bwd(Hq=3, Hkv=2) == 2                   # Hq % Hkv != 0
+    assert bwd(D=96) == 3                          # head size not built
+    assert bwd(causal=0, window=4) == 2            # window is causal only
+    assert bwd(scale=0.0) == 2
+    assert bwd(input_pos=-1) == 2
+    for name in ("dQ", "dK", "dV", "dO", "LSE", "O", "Q"):
+        assert bwd(**{name: None}) == 1, name      # NULL buffer with work to do
+    assert bwd(dQ=ctypes.c_void_p(24)) == 2        # gradients must be 16-byte aligned
+    assert bwd(dK=ctypes.c_void_p(40)) == 2
+    assert bwd(LSE=ctypes.c_void_p(18)) == 2       # LSE must be 4-byte aligned
+    assert bwd(B=0) == 0                           # nothing to do
