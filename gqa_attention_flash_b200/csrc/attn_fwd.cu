@@ -581,20 +581,27 @@ __global__ void __launch_bounds__(kThreads, 1)
                 resc = true;
             }
             const float neg_m = (m_used == neg_inf()) ? 0.f : -m_used;
-            float sum0 = 0.f, sum1 = 0.f;
+            // exponent arguments and the two running sums on packed fp32 pairs (one
+            // f32x2 FMA / add per two scores; same roundings as the scalar forms)
+            const uint64_t sl2x2 = f2_pack(sl2, sl2), negm2 = f2_pack(neg_m, neg_m);
+            uint64_t sum2 = f2_pack(0.f, 0.f);
 #pragma unroll
             for (int c = 0; c < 4; ++c) {
                 uint32_t pk[16];
 #pragma unroll
                 for (int k = 0; k < 16; ++k) {
-                    const float p0 = fast_exp2(fmaf(s[c * 32 + 2 * k], sl2, neg_m));
-                    const float p1 = fast_exp2(fmaf(s[c * 32 + 2 * k + 1], sl2, neg_m));
-                    sum0 += p0;
-                    sum1 += p1;
+                    float x0, x1;
+                    f2_unpack(f2_fma(f2_pack(s[c * 32 + 2 * k], s[c * 32 + 2 * k + 1]), sl2x2, negm2),
+                              x0, x1);
+                    const float p0 = fast_exp2(x0);
+                    const float p1 = fast_exp2(x1);
+                    sum2 = f2_add(sum2, f2_pack(p0, p1));
                     pk[k] = pack_bf16x2(p0, p1);
                 }
                 tmem_st16(s_addr + c * 16, pk);
             }
+            float sum0, sum1;
+            f2_unpack(sum2, sum0, sum1);
             l = l * alpha + (sum0 + sum1);
             // O correction.  S_t(i) completing implies P_t(i-1) V has completed (same
             // issuing thread, in order), so O_t is quiet until we arrive on P_FULL.
