@@ -286,14 +286,14 @@ __global__ void __launch_bounds__(kThreadsTc, 1)
                 const int hq = hkv * p.group + it / n_qt;
                 const int q0 = (qt_lo + it % n_qt) * TB;
                 const long long qrow = (long long)(b * p.Hq + hq) * p.Sq;
-                // the tile's LSE (log2 units) and delta, loaded before the slot is free
+                // the tile's -LSE (log2 units) and -delta, loaded before the slot is free
                 float lr[TB / 32], dr[TB / 32];
 #pragma unroll
                 for (int k = 0; k < TB / 32; ++k) {
                     const int i = q0 + lane + 32 * k;
                     const bool ok = i < p.Sq;
-                    lr[k] = ok ? p.LSE[qrow + i] * kLog2e : ninf();
-                    dr[k] = ok ? p.delta[qrow + i] : 0.f;
+                    lr[k] = ok ? -p.LSE[qrow + i] * kLog2e : -ninf();
+                    dr[k] = ok ? -p.delta[qrow + i] : 0.f;
                 }
                 // dO half: free once dV of the slot's previous item has run
                 if (use > 0 && !warp_wait(bar(C::BAR_EMPTYD + st), (use - 1) & 1, abort_flag,
@@ -399,16 +399,23 @@ __global__ void __launch_bounds__(kThreadsTc, 1)
                 tmem_wait_ld();
                 reg_fence32(sv[0]);
                 reg_fence32(sv[1]);
+                // exponent arguments on packed fp32 pairs (rows[] holds -LSE * log2 e)
                 const float4 *l4 = reinterpret_cast<const float4 *>(rows + cb);
+                const uint64_t sl2x2 = f2_pack(p.scale_log2, p.scale_log2);
 #pragma unroll
                 for (int q = 0; q < 16; ++q) {
                     const float4 l = l4[q];
-                    const float lv[4] = {l.x, l.y, l.z, l.w};
 #pragma unroll
-                    for (int e = 0; e < 4; ++e) {
-                        const int x = 4 * q + e;
-                        const float v = fast_exp2(fmaf(__uint_as_float(sv[x >> 5][x & 31]), p.scale_log2, -lv[e]));
-                        pr[x] = (x >= lo && x < hi) ? v : 0.f;
+                    for (int h = 0; h < 2; ++h) {
+                        const int x = 4 * q + 2 * h;
+                        float x0, x1;
+                        f2_unpack(f2_fma(f2_pack(__uint_as_float(sv[x >> 5][x & 31]),
+                                                 __uint_as_float(sv[x >> 5][(x + 1) & 31])),
+                                         sl2x2, h ? f2_pack(l.z, l.w) : f2_pack(l.x, l.y)),
+                                  x0, x1);
+                        const float v0 = fast_exp2(x0), v1 = fast_exp2(x1);
+                        pr[x] = (x >= lo && x < hi) ? v0 : 0.f;
+                        pr[x + 1] = (x + 1 >= lo && x + 1 < hi) ? v1 : 0.f;
                     }
                 }
             }
@@ -434,15 +441,18 @@ __global__ void __launch_bounds__(kThreadsTc, 1)
                 tmem_wait_ld();
                 reg_fence32(dv[0]);
                 reg_fence32(dv[1]);
+                // dS^T = P^T (dP^T - delta) on packed pairs (rows[TB..] holds -delta)
                 const float4 *d4 = reinterpret_cast<const float4 *>(rows + TB + cb);
 #pragma unroll
                 for (int q = 0; q < 16; ++q) {
                     const float4 dl = d4[q];
-                    const float dlv[4] = {dl.x, dl.y, dl.z, dl.w};
 #pragma unroll
-                    for (int e = 0; e < 4; ++e) {
-                        const int x = 4 * q + e;
-                        pr[x] = pr[x] * (__uint_as_float(dv[x >> 5][x & 31]) - dlv[e]);
+                    for (int h = 0; h < 2; ++h) {
+                        const int x = 4 * q + 2 * h;
+                        const uint64_t t2 = f2_add(f2_pack(__uint_as_float(dv[x >> 5][x & 31]),
+                                                           __uint_as_float(dv[x >> 5][(x + 1) & 31])),
+                                                   h ? f2_pack(dl.z, dl.w) : f2_pack(dl.x, dl.y));
+                        f2_unpack(f2_mul(f2_pack(pr[x], pr[x + 1]), t2), pr[x], pr[x + 1]);
                     }
                 }
             }
@@ -643,10 +653,17 @@ __global__ void __launch_bounds__(kThreadsTc, 1)
                 tmem_wait_ld();
                 reg_fence32(sv[0]);
                 reg_fence32(sv[1]);
+                const uint64_t sl2x2 = f2_pack(p.scale_log2, p.scale_log2), nl2 = f2_pack(-lse2, -lse2);
 #pragma unroll
-                for (int x = 0; x < 64; ++x) {
-                    const float v = fast_exp2(fmaf(__uint_as_float(sv[x >> 5][x & 31]), p.scale_log2, -lse2));
-                    pr[x] = (x >= clo && x < chi) ? v : 0.f;
+                for (int x = 0; x < 64; x += 2) {
+                    float x0, x1;
+                    f2_unpack(f2_fma(f2_pack(__uint_as_float(sv[x >> 5][x & 31]),
+                                             __uint_as_float(sv[x >> 5][(x + 1) & 31])),
+                                     sl2x2, nl2),
+                              x0, x1);
+                    const float v0 = fast_exp2(x0), v1 = fast_exp2(x1);
+                    pr[x] = (x >= clo && x < chi) ? v0 : 0.f;
+                    pr[x + 1] = (x + 1 >= clo && x + 1 < chi) ? v1 : 0.f;
                 }
             }
             if (!warp_wait(bar(C::BAR_DPFULL), g & 1, abort_flag, p.wait_limit_ns, p.status)) {
@@ -664,11 +681,17 @@ __global__ void __launch_bounds__(kThreadsTc, 1)
 #pragma unroll
                 for (int c = 0; c < 2; ++c) {
                     uint32_t pk[16];
+                    const uint64_t nd2 = f2_pack(-del, -del);
 #pragma unroll
                     for (int k = 0; k < 16; ++k) {
                         const int x = 32 * c + 2 * k;
-                        pk[k] = pack_bf16x2(pr[x] * (__uint_as_float(dv[c][2 * k]) - del),
-                                            pr[x + 1] * (__uint_as_float(dv[c][2 * k + 1]) - del));
+                        float d0, d1;
+                        f2_unpack(f2_mul(f2_pack(pr[x], pr[x + 1]),
+                                         f2_add(f2_pack(__uint_as_float(dv[c][2 * k]),
+                                                        __uint_as_float(dv[c][2 * k + 1])),
+                                                nd2)),
+                                  d0, d1);
+                        pk[k] = pack_bf16x2(d0, d1);
                     }
                     tmem_st16(t_s + 16 * c, pk);  // dS over this warp's own S columns
                 }
