@@ -82,6 +82,13 @@ struct TcParams {
 
 __device__ __forceinline__ float ninf() { return __int_as_float(0xff800000); }
 
+// a * b on both fp32 halves of a packed pair (see f2_fma / f2_add).
+__device__ __forceinline__ uint64_t f2_mul(uint64_t a, uint64_t b) {
+    uint64_t d;
+    asm("mul.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+    return d;
+}
+
 __device__ __forceinline__ void tc_lengths(const TcParams &p, int b, int &k_end, int &q_end) {
     k_end = p.Sk;
     q_end = p.Sq;
