@@ -12,16 +12,21 @@
 //              P^T and dP^T into dS^T (bf16, written back over their own columns)
 //              and writes its half of the dK, dV rows
 //   warp 8     TMA: K, V of the tile once, then Q, dO of every (query head of the
-//              group, 128-row query tile that sees the key tile) into a 2-stage
-//              ring; it also copies that tile's LSE and delta next to them
+//              group, 128-row query tile that sees the key tile) into a 2-slot
+//              ring whose Q and dO halves are released separately (after dK and
+//              after dV); it also copies that tile's -LSE (log2 units) and -delta
+//              next to them
 //   warp 9     MMA issuer and TMEM owner
 //   TMEM (512 columns): S^T | dP^T | dV | dK.
 //   Tensor-pipe order per ring item t: dP^T(t), [P^T(t) ready] dV += P^T dO,
 //   S^T(t+1), [dS^T(t) ready] dK += dS^T Q -- so P^T(t+1) is computed while dK(t)
 //   and dP^T(t+1) run, and dS^T(t) while dV(t) and S^T(t+1) run.
 // bwd_dq_tc_kernel: one CTA per (128-row query tile, query head, batch), same
-//   roles over the visible 128-key tiles; TMEM: S | dP | dQ | dS (bf16).  Order:
-//   [S(g) read] S(g+1), [dS(g) ready] dQ += dS K, dP(g+1).
+//   roles over the visible 128-key tiles, Q and dO resident, K in a 3-slot and V
+//   in a 2-slot ring; TMEM: S0 | S1 | dP | dQ, dS (bf16) written over its own S
+//   buffer.  Order: S(0), dP(0), S(1), then per key tile g: [dS(g) ready]
+//   dQ += dS(g) K(g), dP(g+1), S(g+2).
+// The elementwise arithmetic runs on packed fp32 pairs (f32x2 FMA / add / mul).
 // dS is recomputed by the dQ kernel rather than reduced with atomics.  Key,
 // value, query and output-gradient rows past the lengths are read as operands,
 // so they must hold finite values (their weights are exactly zero).
