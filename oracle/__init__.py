@@ -83,6 +83,9 @@ class Oracle:
         L.oracle_attn_bwd.restype = ctypes.c_int
         L.oracle_attn_bwd.argtypes = [_D] * 7 + [ctypes.c_int] * 6 + [
             ctypes.c_double, ctypes.c_int, ctypes.c_int, ctypes.c_int, _I, _I]
+        L.oracle_attn_visible.restype = ctypes.c_int
+        L.oracle_attn_visible.argtypes = [ctypes.c_void_p] + [ctypes.c_int] * 6 + [_I, _I, _I,
+                                                                                 ctypes.c_int]
         L.oracle_decode.restype = ctypes.c_int
         L.oracle_decode.argtypes = [_D, _D, _D, _D, _D] + [ctypes.c_int] * 5 + [_I]
 
@@ -129,6 +132,23 @@ class Oracle:
         if rc != 0:
             raise ValueError("oracle_attn_fwd rejected its arguments")
         return O, LSE
+
+    def attn_visible(self, B, Sq, Sk, causal=False, window=0, input_pos=0, k_lengths=None,
+                     q_lengths=None, rows=None):
+        """uint8 (B, n, Sk): 1 where query row i of batch b sees key j under the
+        masks of attn_fwd (the same mask rows its scores get), else 0.  ``rows``
+        selects absolute query rows (default: all Sq).  The decode key set is
+        ``attn_visible(B, 1, S_cap, k_lengths=lengths)``."""
+        rows_a = _i32(rows)
+        n = Sq if rows_a is None else rows_a.shape[0]
+        kl, ql = _i32(k_lengths), _i32(q_lengths)
+        out = np.empty((B, n, Sk), dtype=np.uint8)
+        rc = self.lib.oracle_attn_visible(out.ctypes.data_as(ctypes.c_void_p), int(B), int(Sq),
+                                          int(Sk), int(causal), int(window), int(input_pos),
+                                          _iptr(kl), _iptr(ql), _iptr(rows_a), n)
+        if rc != 0:
+            raise ValueError("oracle_attn_visible rejected its arguments")
+        return out
 
     # -- Tylo.jl "Primitives" page, flex_attention! -----------------------------------
     def flex_fwd(self, Q, K, V, scale, causal=False, window=0, input_pos=0,

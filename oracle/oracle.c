@@ -149,6 +149,48 @@ static void mask_row(double *m, long i, int Sk, int causal, int window, int inpu
 }
 
 /*
+ * Which keys each requested query row of `attention!` sees: out (B, n_rows, Sk)
+ * uint8 holds 1 where the additive mask of oracle_attn_fwd's score row is 0.0
+ * and 0 where it is -inf -- the same mask_row, so the visible set is exactly the
+ * one whose keys oracle_attn_fwd weighs.  The mask does not depend on the head.
+ * Rows as in oracle_attn_fwd (rows == NULL: all Sq rows).  With Sq = 1,
+ * causal = 0 and k_lengths = the decode lengths it is the key set of
+ * `decode_attention!` (the first lengths[b] cached keys).
+ * Returns 0, or -1 on bad arguments.
+ */
+int oracle_attn_visible(unsigned char *out, int B, int Sq, int Sk, int causal, int window,
+                        int input_pos, const int *k_lengths, const int *q_lengths,
+                        const int *rows, int n_rows) {
+    if (B < 0 || Sq < 0 || Sk < 0) return -1;
+    if (window > 0 && !causal) return -1;
+    if (rows == NULL) n_rows = Sq;
+    const long total = (long)B * n_rows;
+    int bad = 0;
+#pragma omp parallel
+    {
+        double *mask = (double *)malloc(sizeof(double) * (Sk > 0 ? Sk : 1));
+        if (mask == NULL) {
+#pragma omp atomic write
+            bad = 1;
+        }
+#pragma omp for schedule(static)
+        for (long t = 0; t < total; ++t) {
+            if (mask == NULL) continue;
+            const long r = t % n_rows;
+            const long b = t / n_rows;
+            const long i = rows ? rows[r] : r;
+            const int k_len = k_lengths ? k_lengths[b] : Sk;
+            const int q_len = q_lengths ? q_lengths[b] : Sq;
+            mask_row(mask, i, Sk, causal, window, input_pos, k_len, q_len);
+            unsigned char *o = out + t * (long)Sk;
+            for (long j = 0; j < Sk; ++j) o[j] = (mask[j] == 0.0) ? 1 : 0;
+        }
+        free(mask);
+    }
+    return bad ? -1 : 0;
+}
+
+/*
  * Tylo.jl "Primitives" page, `attention!` (+ GQA rule of `flex_attention!`).
  * For every batch b, query head hq and requested query row:
  *   s_j   = scale * <Q_i, K_j> + mask_j          (explicit score row)

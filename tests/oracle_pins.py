@@ -626,7 +626,60 @@ def pin_bwd_gqa_and_uniform(orc):
     assert np.max(np.abs(dV - want)) < 1e-12
 
 
+def pin_visibility(orc):
+    """attn_visible (the key set each row's scores keep) against three things:
+    the page-1 causal_mask / sliding_window_mask of the same shape (visible ⇔
+    entry 0); the keys attn_fwd itself weighs, read off with K = 0 and V = I (O[i,
+    j] ≠ 0 ⇔ key j carries weight), with GQA, lengths, input_pos, a window and
+    a row subset; and the decode key set, the first lengths[b] keys."""
+    for S in range(1, 10):
+        for offset in range(0, 4):
+            vis = orc.attn_visible(1, S, offset + S, causal=True, input_pos=offset)[0]
+            assert np.array_equal(vis == 1, orc.causal_mask(S, offset)[0, 0] == 0.0)
+            for w in range(1, S + offset + 1):
+                vis = orc.attn_visible(1, S, offset + S, causal=True, window=w,
+                                       input_pos=offset)[0]
+                m = orc.sliding_window_mask(S, w, offset)[0, 0]
+                assert np.array_equal(vis == 1, m == 0.0), (S, offset, w)
+    rng = _rng(31)
+    B, Hq, Hkv, Sq, Sk = 3, 4, 2, 9, 13
+    Q = rng.standard_normal((B, Hq, Sq, Sk))
+    K = np.zeros((B, Hkv, Sk, Sk))
+    V = np.broadcast_to(np.eye(Sk), (B, Hkv, Sk, Sk)).copy()
+    k_len = np.array([13, 6, 0], dtype=np.int32)
+    q_len = np.array([9, 4, 9], dtype=np.int32)
+    for causal, window, input_pos, rows in [(False, 0, 0, None), (True, 0, 4, None),
+                                            (True, 3, 2, None), (True, 1, 0, [0, 5, 8]),
+                                            (True, 0, 0, [8, 2])]:
+        kw = dict(causal=causal, window=window, input_pos=input_pos, k_lengths=k_len,
+                  q_lengths=q_len)
+        Qr = Q if rows is None else Q[:, :, rows]
+        O, L = orc.attn_fwd(Qr, K, V, 0.7, rows=rows, Sq=Sq, **kw)
+        vis = orc.attn_visible(B, Sq, Sk, rows=rows, **kw)
+        n_rows = Sq if rows is None else len(rows)
+        assert vis.shape == (B, n_rows, Sk) and vis.dtype == np.uint8
+        assert set(np.unique(vis)) <= {0, 1}
+        for hq in range(Hq):
+            assert np.array_equal(O[:, hq] != 0.0, vis == 1), (causal, window, input_pos, hq)
+        cnt = vis.sum(-1)
+        for b in range(B):
+            for r in range(n_rows):
+                i = r if rows is None else rows[r]
+                if i >= q_len[b]:
+                    want = 0
+                elif causal:
+                    want = _visible_count(input_pos + i, window, int(k_len[b]))
+                else:
+                    want = int(k_len[b])
+                assert cnt[b, r] == want, (b, i)
+    lengths = np.array([0, 1, 7, 20], dtype=np.int32)
+    vis = orc.attn_visible(4, 1, 20, k_lengths=lengths)
+    for b, n in enumerate(lengths):
+        assert np.array_equal(vis[b, 0], (np.arange(20) < n).astype(np.uint8))
+
+
 PINS = [
+    pin_visibility,
     pin_causal_mask_shape_and_rows,
     pin_sliding_window_rows,
     pin_two_key_golden,

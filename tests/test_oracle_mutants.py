@@ -84,6 +84,13 @@ MUTANTS = {
     "bwd_dv_from_ds": ("dVh[j * D + d] += prob[j] * go[d];", "dVh[j * D + d] += ds * go[d];"),
     "bwd_one_head_per_group": ("for (long hq = hkv * group; hq < (hkv + 1) * group; ++hq)",
                                "for (long hq = hkv * group; hq < hkv * group + 1; ++hq)"),
+    "visible_inverted": ("o[j] = (mask[j] == 0.0) ? 1 : 0;", "o[j] = (mask[j] == 0.0) ? 0 : 1;"),
+    "visible_batch_stride": ("unsigned char *o = out + t * (long)Sk;",
+                             "unsigned char *o = out + r * (long)Sk;"),
+    "visible_window_dropped": ("mask_row(mask, i, Sk, causal, window, input_pos, k_len, q_len);\n"
+                               "            unsigned char",
+                               "mask_row(mask, i, Sk, causal, 0, input_pos, k_len, q_len);\n"
+                               "            unsigned char"),
     "bwd_mask_ignored": ("mask_row(mrow, i, Sk, causal, window, input_pos, k_len, q_len);",
                          "mask_row(mrow, i, Sk, 0, 0, input_pos, Sk, Sq);"),
 }
@@ -103,10 +110,11 @@ def test_mutant_is_caught(name, source, tmp_path):
     src.write_text(source.replace(old, new))
     lib = oracle.build(str(src), str(tmp_path / f"lib{name}.so"))
     mutant = oracle.Oracle(lib)
-    failed = []
-    for pin in PINS:
+    failed = None
+    for pin in PINS:  # one failing pin is enough; stop at the first
         try:
             pin(mutant)
         except AssertionError:
-            failed.append(pin.__name__)
+            failed = pin.__name__
+            break
     assert failed, f"no pin catches the planted mistake {name}"
