@@ -28,8 +28,11 @@
 //   dQ += dS(g) K(g), dP(g+1), S(g+2).
 // The elementwise arithmetic runs on packed fp32 pairs (f32x2 FMA / add / mul).
 // dS is recomputed by the dQ kernel rather than reduced with atomics.  Key,
-// value, query and output-gradient rows past the lengths are read as operands,
-// so they must hold finite values (their weights are exactly zero).
+// value, query and output-gradient rows past the lengths are read as MMA
+// operands with weight exactly zero, so they must hold finite values: zero times
+// NaN or Inf is NaN, which would reach the gradients of valid rows.  The rows of
+// dQ past q_lengths and of dK, dV past k_lengths are themselves written as +0.0
+// by selection.
 #include <cuda_bf16.h>
 
 #include "internal.h"
@@ -212,17 +215,21 @@ __device__ __forceinline__ void tc_teardown(uint8_t *smem, uint32_t tmem) {
 // times `mul`, as bf16 to dst[c0 ..).
 template <int D>
 __device__ __forceinline__ void tc_store_half(uint32_t taddr, __nv_bfloat16 *dst, int c0, float mul,
-                                              bool store) {
+                                              bool store, bool valid) {
 #pragma unroll
     for (int c = 0; c < D / 64; ++c) {
         uint32_t v[32];
         tmem_ld32(taddr + c0 + c * 32, v);
         tmem_wait_ld();
         reg_fence32(v);
+        // rows past the lengths are +0.0 by selection (their accumulators saw
+        // only zero weights, but zero times a non-finite operand is NaN)
         uint32_t o16[16];
 #pragma unroll
         for (int k = 0; k < 16; ++k)
-            o16[k] = pack_bf16x2(__uint_as_float(v[2 * k]) * mul, __uint_as_float(v[2 * k + 1]) * mul);
+            o16[k] = valid ? pack_bf16x2(__uint_as_float(v[2 * k]) * mul,
+                                         __uint_as_float(v[2 * k + 1]) * mul)
+                           : 0u;
         if (store) {
             uint4 *d4 = reinterpret_cast<uint4 *>(dst + c0 + c * 32);
 #pragma unroll
@@ -484,8 +491,10 @@ __global__ void __launch_bounds__(kThreadsTc, 1)
         const long long krow = (long long)(b * p.Hkv + hkv) * p.Sk + j;
         if (have) {
             tc_fence_after();
-            tc_store_half<D>(trow + C::COL_A, p.dV + krow * D, half * (D / 2), 1.f, j < p.Sk);
-            tc_store_half<D>(trow + C::COL_B, p.dK + krow * D, half * (D / 2), p.scale, j < p.Sk);
+            tc_store_half<D>(trow + C::COL_A, p.dV + krow * D, half * (D / 2), 1.f, j < p.Sk,
+                             j < k_end);
+            tc_store_half<D>(trow + C::COL_B, p.dK + krow * D, half * (D / 2), p.scale, j < p.Sk,
+                             j < k_end);
         } else if (j < p.Sk && !*abort_flag) {
             tc_zero_half<D>(p.dV + krow * D, half * (D / 2));
             tc_zero_half<D>(p.dK + krow * D, half * (D / 2));
@@ -716,7 +725,8 @@ __global__ void __launch_bounds__(kThreadsTc, 1)
                           warp_wait(bar(C::BAR_DONE), 0, abort_flag, p.wait_limit_ns, p.status);
         if (have) {
             tc_fence_after();
-            tc_store_half<D>(trow + C::COL_DQ, p.dQ + (qrow + i) * D, half * (D / 2), p.scale, i < p.Sq);
+            tc_store_half<D>(trow + C::COL_DQ, p.dQ + (qrow + i) * D, half * (D / 2), p.scale, i < p.Sq,
+                             i < q_end);
         } else if (i < p.Sq && !*abort_flag) {
             tc_zero_half<D>(p.dQ + (qrow + i) * D, half * (D / 2));
         }

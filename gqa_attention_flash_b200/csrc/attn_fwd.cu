@@ -664,11 +664,15 @@ __global__ void __launch_bounds__(kThreads, 1)
                 tmem_ld32(o_addr + c * 32, v);
                 tmem_wait_ld();
                 reg_fence32(v);
+                // Rows past q_lengths ran the whole chain on whatever the padding of
+                // Q holds (NaN included); their output is selected, not scaled, to
+                // +0.0 so nothing of that padding reaches O.
                 uint32_t o16[16];
 #pragma unroll
                 for (int k = 0; k < 16; ++k)
-                    o16[k] = pack_bf16x2(__uint_as_float(v[2 * k]) * inv_l,
-                                         __uint_as_float(v[2 * k + 1]) * inv_l);
+                    o16[k] = out_valid ? pack_bf16x2(__uint_as_float(v[2 * k]) * inv_l,
+                                                     __uint_as_float(v[2 * k + 1]) * inv_l)
+                                       : 0u;
                 if (row_in) {
                     uint4 *dst = reinterpret_cast<uint4 *>(orow + c * 32);
 #pragma unroll

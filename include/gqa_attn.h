@@ -87,8 +87,9 @@ attn_status_t attn_fwd(void *O, const void *Q, const void *K, const void *V, flo
  *
  * Same definition and arguments as attn_fwd, with q_lengths an int32 (B,)
  * device array or NULL (= Sq): query rows i >= q_lengths[b] are invalid and
- * get O = 0 and LSE = -inf (Tylo.jl "Primitives" page, entry `attention!`,
- * keyword q_lengths).  attn_fwd(...) is attn_fwd_varlen(..., q_lengths=NULL).
+ * get O = +0.0 (every bit zero) and LSE = -inf, whatever those rows of Q hold,
+ * NaN and Inf included (Tylo.jl "Primitives" page, entry `attention!`, keyword
+ * q_lengths).  attn_fwd(...) is attn_fwd_varlen(..., q_lengths=NULL).
  */
 attn_status_t attn_fwd_varlen(void *O, const void *Q, const void *K, const void *V, float *LSE,
                               int B, int Hq, int Hkv, int Sq, int Sk, int D, float scale,
@@ -147,8 +148,11 @@ attn_status_t attn_fwd_flex(void *O, const void *Q, const void *K, const void *V
  * With P = exp(scale Q K^T - LSE) on the visible pairs: dV = P^T dO,
  * dS = P (dO V^T - rowsum(dO O)), dQ = scale dS K, dK = scale dS^T Q; dK / dV
  * of a KV head sum over the query heads it serves; keys never visible and
- * query rows past q_lengths get zero gradients.  Allocates a stream-ordered
- * workspace of B * Hq * Sq floats.  Errors as attn_fwd.
+ * query rows past q_lengths get zero gradients (rows of dQ past q_lengths and
+ * of dK, dV past k_lengths are +0.0).  Padding rows (Q, dO, O past q_lengths;
+ * K, V past k_lengths) must hold finite values: they enter the tensor-core
+ * products with weight zero, and zero times NaN or Inf is NaN.  Allocates a
+ * stream-ordered workspace of B * Hq * Sq floats.  Errors as attn_fwd.
  */
 attn_status_t attn_bwd(void *dQ, void *dK, void *dV, const void *dO, const void *Q, const void *K,
                        const void *V, const void *O, const float *LSE, int B, int Hq, int Hkv,

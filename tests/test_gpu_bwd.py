@@ -94,6 +94,35 @@ def test_backward_masked_rows_and_keys_are_zero():
     assert torch.all(dQ[0, :, 90:] == 0)
 
 
+def test_backward_finite_padding(orc):
+    """Padding rows may hold any finite value (the documented limit: they enter the
+    tensor-core products with weight zero, so they must not be NaN or Inf): Q and
+    dO rows past q_lengths and K, V rows past k_lengths hold +-3e4, and the
+    gradients still match the oracle's (computed from the clean tensors) with the
+    padded rows of dQ, dK, dV exactly +0.0."""
+    B, Hq, Hkv, S, D = 2, 4, 2, 333, 128
+    Q, K, V = W.random_prefill(91, B, Hq, Hkv, S, S, D)
+    dO = torch.randn(B, Hq, S, D, generator=torch.Generator().manual_seed(9)).to(torch.bfloat16)
+    kl = torch.tensor([333, 190], dtype=torch.int32)
+    ql = torch.tensor([250, 333], dtype=torch.int32)
+    Qp, Kp, Vp, dOp = Q.clone(), K.clone(), V.clone(), dO.clone()
+    Qp[0, :, 250:] = 3e4
+    dOp[0, :, 250:] = -3e4
+    Kp[1, :, 190:] = -3e4
+    Vp[1, :, 190:] = 3e4
+    scale = 1.0 / math.sqrt(D)
+    dQ, dK, dV = gpu_fwd_bwd(Qp, Kp, Vp, dOp, scale, True, 0, 0, kl, ql)
+    rQ, rK, rV = orc.attn_bwd(Q.double().numpy(), K.double().numpy(), V.double().numpy(),
+                              dO.double().numpy(), scale, causal=True, k_lengths=kl.numpy(),
+                              q_lengths=ql.numpy())
+    check(dQ, rQ, "dQ finite padding")
+    check(dK, rK, "dK finite padding")
+    check(dV, rV, "dV finite padding")
+    assert torch.all(dQ[0, :, 250:].view(torch.int16) == 0)
+    assert torch.all(dK[1, :, 190:].view(torch.int16) == 0)
+    assert torch.all(dV[1, :, 190:].view(torch.int16) == 0)
+
+
 def test_backward_full_size_llm(orc):
     """The LLM causal shape (B4 Hq32 Hkv8 S4096 D128) as the benchmark runs it:
     dQ on sampled rows and dK / dV on sampled keys of one batch entry, against the

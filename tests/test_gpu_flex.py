@@ -183,3 +183,32 @@ def test_full_size_flex_workloads(orc, key):
                           doc_q=None if doc is None else doc.numpy(),
                           doc_kv=None if doc is None else doc.numpy())
     compare(O, L, Or, Lr, rows=rows, what=f"full-size {key}")
+
+
+@pytest.mark.parametrize("mod", ["softcap", "alibi", "document"])
+def test_nan_q_rows_past_q_lengths(orc, mod):
+    """flex_attention! instantiations (soft cap, ALiBi, the document-mask list
+    path): NaN query rows past q_lengths give O = +0.0 and LSE = -inf, and the
+    valid rows match the oracle."""
+    from gqa_attention_flash_b200 import binding
+    B, Hq, Hkv, S, D = 2, 4, 2, 390, 128
+    Q, K, V = W.random_prefill(51, B, Hq, Hkv, S, S, D)
+    ql = torch.tensor([390, 200], dtype=torch.int32)
+    kl = torch.tensor([390, 390], dtype=torch.int32)
+    Qp = Q.clone()
+    Qp[1, :, 200:] = float("nan")
+    kw = {}
+    if mod == "softcap":
+        kw = dict(softcap=5.0)
+    elif mod == "alibi":
+        kw = dict(alibi=W.alibi_slopes(Hq, seed=5))
+    else:
+        doc = W.document_ids(S, seed=6, min_len=20, max_len=150)
+        kw = dict(doc_q=doc, doc_kv=doc)
+    bm = binding.block_mask_document(S, S, kw["doc_q"], kw["doc_kv"], True, 0) \
+        if mod == "document" else None
+    O, L = gpu_flex(Qp, K, V, 0.09, True, 0, 0, kl, ql, block_mask=bm, **kw)
+    Or, Lr = oracle_flex(orc, Q, K, V, 0.09, True, 0, 0, kl, ql, **kw)
+    compare(O, L, Or, Lr, what=f"flex {mod} NaN past q_len")
+    assert torch.all(O[1, :, 200:].view(torch.int16) == 0)
+    assert torch.all(torch.isneginf(L[1, :, 200:]))

@@ -121,3 +121,51 @@ def test_running_max_jumps(orc, causal):
     O, L = gpu_prefill(Q, K, V, scale, causal)
     Or, Lr = oracle_prefill(orc, Q, K, V, scale, causal)
     compare(O, L, Or, Lr, what=f"max jumps causal={causal}")
+
+
+@pytest.mark.parametrize("D,poison", [(128, float("nan")), (64, float("inf"))])
+def test_non_finite_q_rows_past_q_lengths(orc, D, poison):
+    """Query rows past q_lengths may hold anything (uninitialised padding, NaN,
+    Inf): their O rows are +0.0 in every bit and their LSE is -inf, and the valid
+    rows still match the oracle (which gets the clean Q)."""
+    B, Hq, Hkv, S = 3, 4, 2, 300
+    Q, K, V = W.random_prefill(13, B, Hq, Hkv, S, S, D)
+    ql = torch.tensor([300, 131, 7], dtype=torch.int32)
+    kl = torch.tensor([300, 250, 300], dtype=torch.int32)
+    Qp = Q.clone()
+    for b, n in enumerate(ql.tolist()):
+        Qp[b, :, n:] = poison
+    for causal, window, input_pos in [(False, 0, 0), (True, 0, 0), (True, 50, 20)]:
+        O, L = gpu_prefill(Qp, K, V, 0.09, causal, window, input_pos, kl, ql)
+        Or, Lr = oracle_prefill(orc, Q, K, V, 0.09, causal, window, input_pos, kl, ql)
+        compare(O, L, Or, Lr, what=f"poisoned Q {causal} {window} {input_pos}")
+        for b, n in enumerate(ql.tolist()):
+            assert torch.all(O[b, :, n:].view(torch.int16) == 0), (b, causal, window)
+            assert torch.all(torch.isneginf(L[b, :, n:]))
+
+
+def test_window_workload_finite_poison(orc):
+    """Probe (ii) on the sliding-window workload at full size: every key and value
+    row past k_lengths holds the finite value 1e4 and every query row past
+    q_lengths holds NaN.  A masked key that leaked into a row would move it by far
+    more than the tolerance; the padded rows must be +0.0 / -inf."""
+    w = W.WINDOW
+    x = W.make_prefill(w)
+    Qp, Kp, Vp = x.Q.clone(), x.K.clone(), x.V.clone()
+    for b, n in enumerate(x.k_lengths.tolist()):
+        Kp[b, :, n:] = 1e4
+        Vp[b, :, n:] = 1e4
+    for b, n in enumerate(x.q_lengths.tolist()):
+        Qp[b, :, n:] = float("nan")
+    O, L = gpu_prefill(Qp, Kp, Vp, w.scale, w.causal, w.window, w.input_pos, x.k_lengths,
+                       x.q_lengths)
+    extra = []
+    for v in x.k_lengths.tolist():
+        extra += [v - 129, v - 128, v - 2, v - 1, v, v + 1, v - w.window, v - w.window + 1]
+    rows = sample_rows(w.Sq, 9, n_random=24, extra=extra)
+    Or, Lr = oracle_prefill(orc, x.Q, x.K, x.V, w.scale, w.causal, w.window, w.input_pos,
+                            x.k_lengths, x.q_lengths, rows=rows)
+    compare(O, L, Or, Lr, rows=rows, what="window poison")
+    for b, n in enumerate(x.q_lengths.tolist()):
+        assert torch.all(O[b, :, n:].view(torch.int16) == 0)
+        assert torch.all(torch.isneginf(L[b, :, n:]))
