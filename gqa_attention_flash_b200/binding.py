@@ -70,6 +70,51 @@ def _ptr(t):
     return None if t is None else ctypes.c_void_p(t.data_ptr())
 
 
+# The C ABI sees raw pointers and sizes only: it cannot tell a transposed view, a
+# float16 tensor or a tensor on another device from the layout it expects.  The
+# wrappers therefore refuse such tensors here, before any call into the library.
+def _tensor(t, name, dtype, shape):
+    """Check dtype, shape (entries of None are free) and row-major contiguity;
+    returns the shape."""
+    if not isinstance(t, torch.Tensor):
+        raise TypeError(f"{name} must be a torch.Tensor, got {type(t).__name__}")
+    if t.dtype != dtype:
+        raise TypeError(f"{name} must be {dtype}, got {t.dtype}")
+    if t.dim() != len(shape) or any(w is not None and w != g for g, w in zip(t.shape, shape)):
+        want = "(" + ", ".join("*" if w is None else str(w) for w in shape) + ")"
+        raise ValueError(f"{name} has shape {tuple(t.shape)}, expected {want}")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous (row-major); call .contiguous()")
+    return tuple(t.shape)
+
+
+def _same_device(**tensors):
+    """Every given tensor on the current CUDA device (the one whose stream the
+    kernels are launched on)."""
+    for name, t in tensors.items():
+        if t is None:
+            continue
+        if not t.is_cuda:
+            raise ValueError(f"{name} must be a CUDA tensor, got device {t.device}")
+        if t.device.index != torch.cuda.current_device():
+            raise ValueError(f"{name} is on {t.device}, but the current device is "
+                             f"cuda:{torch.cuda.current_device()}")
+
+
+def _check_prefill(O, Q, K, V, LSE, k_lengths, q_lengths):
+    B, Hq, Sq, D = _tensor(Q, "Q", torch.bfloat16, (None,) * 4)
+    _, Hkv, Sk, _ = _tensor(K, "K", torch.bfloat16, (B, None, None, D))
+    _tensor(V, "V", torch.bfloat16, (B, Hkv, Sk, D))
+    _tensor(O, "O", torch.bfloat16, (B, Hq, Sq, D))
+    if LSE is not None:
+        _tensor(LSE, "LSE", torch.float32, (B, Hq, Sq))
+    if k_lengths is not None:
+        _tensor(k_lengths, "k_lengths", torch.int32, (B,))
+    if q_lengths is not None:
+        _tensor(q_lengths, "q_lengths", torch.int32, (B,))
+    return B, Hq, Hkv, Sq, Sk, D
+
+
 def _stream(stream):
     if stream is None:
         stream = torch.cuda.current_stream()
@@ -92,8 +137,8 @@ def attn_fwd(O, Q, K, V, LSE, scale, causal=False, window=0, input_pos=0, k_leng
     Shapes are read from the tensors: Q (B,Hq,Sq,D), K/V (B,Hkv,Sk,D).  Calls
     ``attn_fwd_varlen`` when q_lengths is given, else ``attn_fwd``.
     """
-    B, Hq, Sq, D = Q.shape
-    _, Hkv, Sk, _ = K.shape
+    B, Hq, Hkv, Sq, Sk, D = _check_prefill(O, Q, K, V, LSE, k_lengths, q_lengths)
+    _same_device(O=O, Q=Q, K=K, V=V, LSE=LSE, k_lengths=k_lengths, q_lengths=q_lengths)
     args = [_ptr(O), _ptr(Q), _ptr(K), _ptr(V), _ptr(LSE), B, Hq, Hkv, Sq, Sk, D, float(scale),
             int(causal), int(window), int(input_pos), _ptr(k_lengths)]
     if q_lengths is not None:
@@ -111,8 +156,19 @@ def attn_fwd_flex(O, Q, K, V, LSE, scale, causal=False, window=0, input_pos=0, k
     AliBiScore (alibi_slopes, fp32 (Hq,)), DocumentMask (doc_q int32 (Sq,), doc_kv
     int32 (Sk,)) and a BlockMask (uint8 (ceil(Sq/64), ceil(Sk/64)), or one per
     (batch, query head) as a 4-D (B, Hq, ., .) tensor), all on the device."""
-    B, Hq, Sq, D = Q.shape
-    _, Hkv, Sk, _ = K.shape
+    B, Hq, Hkv, Sq, Sk, D = _check_prefill(O, Q, K, V, LSE, k_lengths, q_lengths)
+    if alibi_slopes is not None:
+        _tensor(alibi_slopes, "alibi_slopes", torch.float32, (Hq,))
+    if doc_q is not None:
+        _tensor(doc_q, "doc_q", torch.int32, (Sq,))
+    if doc_kv is not None:
+        _tensor(doc_kv, "doc_kv", torch.int32, (Sk,))
+    if block_mask is not None:
+        nqb, nkb = block_mask_shape(Sq, Sk)
+        _tensor(block_mask, "block_mask", torch.uint8,
+                (B, Hq, nqb, nkb) if block_mask.dim() == 4 else (nqb, nkb))
+    _same_device(O=O, Q=Q, K=K, V=V, LSE=LSE, k_lengths=k_lengths, q_lengths=q_lengths,
+                 alibi_slopes=alibi_slopes, doc_q=doc_q, doc_kv=doc_kv, block_mask=block_mask)
     rc = lib.attn_fwd_flex(_ptr(O), _ptr(Q), _ptr(K), _ptr(V), _ptr(LSE), B, Hq, Hkv, Sq, Sk, D,
                            float(scale), int(causal), int(window), int(input_pos),
                            _ptr(k_lengths), _ptr(q_lengths), float(softcap), _ptr(alibi_slopes),
@@ -126,8 +182,9 @@ def rbs_block_mask(Q, K, alpha_base=0.22, alpha_rescue=0.18, diagonal=1, want_sc
                    stream=None):
     """Block-sparse prefill mask from the RBS block scores: uint8 (B, Hq, nqb, nkb)
     device tensor (2 = keep, 0 = skip), plus the (base, rescue) scores if asked."""
-    B, Hq, Sq, D = Q.shape
-    _, Hkv, Sk, _ = K.shape
+    B, Hq, Sq, D = _tensor(Q, "Q", torch.bfloat16, (None,) * 4)
+    _, Hkv, Sk, _ = _tensor(K, "K", torch.bfloat16, (B, None, None, D))
+    _same_device(Q=Q, K=K)
     shape = (B, Hq, (Sq + 63) // 64, (Sk + 63) // 64)
     mask = torch.empty(shape, dtype=torch.uint8, device=Q.device)
     base = torch.empty(shape, dtype=torch.float32, device=Q.device) if want_scores else None
@@ -143,8 +200,15 @@ def attn_bwd(dQ, dK, dV, dO, Q, K, V, O, LSE, scale, causal=False, window=0, inp
              k_lengths=None, q_lengths=None, stream=None):
     """Backward of attn_fwd: fill dQ (like Q) and dK, dV (like K, V) in place from dO,
     the forward's inputs, output O and LSE."""
-    B, Hq, Sq, D = Q.shape
-    _, Hkv, Sk, _ = K.shape
+    B, Hq, Hkv, Sq, Sk, D = _check_prefill(O, Q, K, V, LSE, k_lengths, q_lengths)
+    if LSE is None:
+        raise ValueError("LSE (the forward's saved statistics) is required")
+    _tensor(dO, "dO", torch.bfloat16, (B, Hq, Sq, D))
+    _tensor(dQ, "dQ", torch.bfloat16, (B, Hq, Sq, D))
+    _tensor(dK, "dK", torch.bfloat16, (B, Hkv, Sk, D))
+    _tensor(dV, "dV", torch.bfloat16, (B, Hkv, Sk, D))
+    _same_device(dQ=dQ, dK=dK, dV=dV, dO=dO, Q=Q, K=K, V=V, O=O, LSE=LSE, k_lengths=k_lengths,
+                 q_lengths=q_lengths)
     rc = lib.attn_bwd(_ptr(dQ), _ptr(dK), _ptr(dV), _ptr(dO), _ptr(Q), _ptr(K), _ptr(V), _ptr(O),
                       _ptr(LSE), B, Hq, Hkv, Sq, Sk, D, float(scale), int(causal), int(window),
                       int(input_pos), _ptr(k_lengths), _ptr(q_lengths), _stream(stream))
@@ -178,10 +242,19 @@ def block_mask_build(Sq, Sk, keep, input_pos=0):
     return out
 
 
+def _check_decode(O, Q, K, V, lengths):
+    B, Hq, D = _tensor(Q, "Q", torch.bfloat16, (None,) * 3)
+    _, Hkv, S_cap, _ = _tensor(K, "K", torch.bfloat16, (B, None, None, D))
+    _tensor(V, "V", torch.bfloat16, (B, Hkv, S_cap, D))
+    _tensor(O, "O", torch.bfloat16, (B, Hq, D))
+    _tensor(lengths, "lengths", torch.int32, (B,))
+    _same_device(O=O, Q=Q, K=K, V=V, lengths=lengths)
+    return B, Hq, Hkv, S_cap, D
+
+
 def attn_decode(O, Q, K, V, lengths, n_splits=8, stream=None):
     """Fill O (B,Hq,D) bf16 in place; Q (B,Hq,D), K/V caches (B,Hkv,S_cap,D)."""
-    B, Hq, D = Q.shape
-    _, Hkv, S_cap, _ = K.shape
+    B, Hq, Hkv, S_cap, D = _check_decode(O, Q, K, V, lengths)
     rc = lib.attn_decode(_ptr(O), _ptr(Q), _ptr(K), _ptr(V), _ptr(lengths), int(n_splits),
                          _stream(stream), B, Hq, Hkv, S_cap, D)
     _check(rc, "attn_decode")
@@ -190,8 +263,15 @@ def attn_decode(O, Q, K, V, lengths, n_splits=8, stream=None):
 def attn_decode_paged(O, Q, K_cache, V_cache, block_tables, seq_lens, n_splits=8, stream=None):
     """Decode from a paged cache: Q (B,Hq,D); K/V caches (num_blocks, block_size, Hkv, D);
     block_tables int32 (B, max_blocks); seq_lens int32 (B,); O (B,Hq,D) filled in place."""
-    B, Hq, D = Q.shape
-    num_blocks, block_size, Hkv, _ = K_cache.shape
+    B, Hq, D = _tensor(Q, "Q", torch.bfloat16, (None,) * 3)
+    num_blocks, block_size, Hkv, _ = _tensor(K_cache, "K_cache", torch.bfloat16,
+                                             (None, None, None, D))
+    _tensor(V_cache, "V_cache", torch.bfloat16, (num_blocks, block_size, Hkv, D))
+    _tensor(O, "O", torch.bfloat16, (B, Hq, D))
+    _tensor(block_tables, "block_tables", torch.int32, (B, None))
+    _tensor(seq_lens, "seq_lens", torch.int32, (B,))
+    _same_device(O=O, Q=Q, K_cache=K_cache, V_cache=V_cache, block_tables=block_tables,
+                 seq_lens=seq_lens)
     rc = lib.attn_decode_paged(_ptr(O), _ptr(Q), _ptr(K_cache), _ptr(V_cache), _ptr(block_tables),
                                _ptr(seq_lens), int(n_splits), _stream(stream), B, Hq, Hkv,
                                num_blocks, block_size, int(block_tables.shape[1]), D)
@@ -202,8 +282,7 @@ def attn_decode_noalloc(O, Q, K, V, lengths, n_splits=8, stream=None):
     """attn_decode without any allocation: the workspace lives in the library's
     fixed 16 MiB device array (for callers that cannot allocate device memory;
     calls that overlap on the GPU share that array and must be ordered)."""
-    B, Hq, D = Q.shape
-    _, Hkv, S_cap, _ = K.shape
+    B, Hq, Hkv, S_cap, D = _check_decode(O, Q, K, V, lengths)
     rc = lib.attn_decode_noalloc(_ptr(O), _ptr(Q), _ptr(K), _ptr(V), _ptr(lengths),
                                  int(n_splits), _stream(stream), B, Hq, Hkv, S_cap, D)
     _check(rc, "attn_decode_noalloc")
