@@ -341,6 +341,11 @@ __global__ void __launch_bounds__(kDecThreads)
                 dst[d] = acc / lsum;
                 if (d == 0) dst[D] = (M + __log2f(lsum)) * 0.69314718055994531f;
             }
+        } else {
+            // A bounded wait ran out: the slice weighs nothing in the combine, so
+            // whatever the workspace held before (another call's partials) never
+            // reaches O.
+            for (int h = threadIdx.x; h < G; h += 32 * kConsumers) ws_base[h * ws_head + D] = neg_inf();
         }
     }
     if (*abort_flag) drain_delay(2000000);

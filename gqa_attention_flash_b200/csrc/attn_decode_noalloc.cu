@@ -16,7 +16,9 @@
 //     different host threads without ordering) race on it and must be
 //     serialised by the caller, e.g. by issuing them on one stream;
 //   - it keeps whatever the last call left; the split kernel writes every
-//     entry the combine kernel reads, so nothing needs clearing between calls.
+//     entry the combine kernel reads (an empty slice, or one whose bounded wait
+//     ran out, writes a log-sum-exp of -inf and so weighs nothing), so nothing
+//     needs clearing between calls.
 // In host code the array's name is only a host-side stand-in, so its device
 // address is looked up with cudaGetSymbolAddress, once per device, on the first
 // call made while that device is current; that first call should come before

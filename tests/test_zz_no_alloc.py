@@ -51,16 +51,37 @@ def test_noalloc_matches_allocating_decode_twice():
         assert d <= O_TOL, (seed, d)
 
 
-def test_noalloc_full_decode_shape_fits():
-    """The benchmark's decode shape (B64 Hq32 n_splits 8 D128: 8.65 MB of
-    workspace) fits in the fixed array."""
+def test_noalloc_same_shape_shorter_lengths():
+    """Two calls of one shape in a row: the first with long sequences fills every
+    slice of the shared array; the second, with much shorter sequences, leaves
+    most slices empty.  Those slices still hold the first call's partials, and
+    they must not reach the second call's output."""
     from gqa_attention_flash_b200 import binding
     lib = binding.lib
+    B, Hq, Hkv, S_cap, D, n_splits = 4, 16, 4, 4096, 128, 8
+    Q, K, V, _ = _inputs(5, B, Hq, Hkv, S_cap, D)
+    for lens in ([4096, 4000, 3900, 4096], [1, 65, 130, 0]):
+        lengths = torch.tensor(lens, dtype=torch.int32, device=Q.device)
+        ref = torch.empty_like(Q)
+        assert _call(lib.attn_decode, ref, Q, K, V, lengths, n_splits) == 0
+        out = torch.full_like(Q, float("nan"))
+        assert _call(lib.attn_decode_noalloc, out, Q, K, V, lengths, n_splits) == 0
+        assert binding.last_device_status() == 0
+        assert torch.all(torch.isfinite(out.float()))
+        d = float((out.float() - ref.float()).abs().max())
+        assert d <= O_TOL, (lens, d)
+    assert torch.all(out[3] == 0)  # length 0: no slice has a key
+
+
+def test_noalloc_full_decode_shape_fits():
+    """The benchmark's decode shape (B64 Hq32 n_splits 8 D128: 8.65 MB of
+    workspace) fits in the fixed array; called through the Python wrapper."""
+    from gqa_attention_flash_b200 import binding
     Q, K, V, lengths = _inputs(3, 64, 32, 8, 256, 128)
     ref = torch.empty_like(Q)
     out = torch.empty_like(Q)
-    assert _call(lib.attn_decode, ref, Q, K, V, lengths, 8) == 0
-    assert _call(lib.attn_decode_noalloc, out, Q, K, V, lengths, 8) == 0
+    binding.attn_decode(ref, Q, K, V, lengths, 8)
+    binding.attn_decode_noalloc(out, Q, K, V, lengths, 8)
     assert binding.last_device_status() == 0
     assert float((out.float() - ref.float()).abs().max()) <= O_TOL
 
