@@ -304,6 +304,8 @@ def time_e2e(step, steps, warmup):
 # CPU oracle timing (cpu_baseline leg and the reference arm)
 # ----------------------------------------------------------------------------------
 def oracle_sample_prefill(orc, w, x, row_stride):
+    """Time the oracle on the query rows i % row_stride == 0 (all batches and
+    heads); returns (algorithmic FLOPs of those rows, seconds, number of rows)."""
     rows = np.arange(0, w.Sq, row_stride, dtype=np.int32)
     Qs = x.Q[:, :, torch.as_tensor(rows, dtype=torch.long)].double().numpy()
     Kd, Vd = x.K.double().numpy(), x.V.double().numpy()
@@ -316,7 +318,10 @@ def oracle_sample_prefill(orc, w, x, row_stride):
     pairs = 0
     for b in range(w.B):
         k_len = int(kl[b]) if kl is not None else w.Sk
+        q_len = int(ql[b]) if ql is not None else w.Sq
         for i in rows:
+            if i >= q_len:
+                continue
             p = w.input_pos + int(i)
             hi = min(k_len, p + 1) if w.causal else k_len
             lo = max(0, p - w.window + 1) if w.window > 0 else 0
@@ -401,6 +406,82 @@ def time_flex(dev, steps, warmup, peak):
                                  if "attn_fwd_kernel_flex_" + key in KERNEL_SOURCES else None,
                                  "kernel": "attn_fwd_kernel<128, flex>"}}
         del Qd, Kd, Vd, O, LSE
+        torch.cuda.empty_cache()
+    return out
+
+
+class L2Flush:
+    """Writes a buffer twice the size of L2 (126 MB) so that the next timed launch
+    starts with none of its inputs in L2."""
+
+    def __init__(self, dev):
+        self.buf = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+
+    def __call__(self):
+        self.buf.fill_(1)
+
+
+def time_prefill_configs(dev, steps, warmup, peak, with_cpu):
+    """The other prefill workloads, each launched alone with inputs resident in HBM
+    and L2 flushed before every timed launch (CUDA events around each launch):
+      window  sliding window 4096 with ragged lengths (attn_fwd_varlen),
+      image   non-causal 64x64-token image attention,
+      tiny    the small causal GQA case, reported as latency per launch.
+    TFLOP/s counts 4 * D * visible (query, key) pairs of the drawn lengths."""
+    from gqa_attention_flash_b200 import binding
+    flush = L2Flush(dev)
+    orc = None
+    if with_cpu:
+        import oracle
+        orc = oracle.default()
+    out = {}
+    for key in ("window", "image", "tiny"):
+        w = W.PREFILL_WORKLOADS[key]
+        x = W.make_prefill(w)
+        Q, K, V = x.Q.to(dev), x.K.to(dev), x.V.to(dev)
+        kl = None if x.k_lengths is None else x.k_lengths.to(dev)
+        ql = None if x.q_lengths is None else x.q_lengths.to(dev)
+        O = torch.empty_like(Q)
+        LSE = torch.empty(Q.shape[:3], dtype=torch.float32, device=dev)
+
+        def run():
+            binding.attn_fwd(O, Q, K, V, LSE, w.scale, w.causal, w.window, w.input_pos, kl, ql)
+        for _ in range(warmup):
+            run()
+        torch.cuda.synchronize()
+        ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+              for _ in range(steps)]
+        for e0, e1 in ev:
+            flush()
+            e0.record()
+            run()
+            e1.record()
+        torch.cuda.synchronize()
+        st = binding.last_device_status()
+        if st != 0:
+            raise RuntimeError(f"{key} device status: {binding.status_string(st)}")
+        ms = sum(a.elapsed_time(b) for a, b in ev) / steps
+        flops = w.flops(x.k_lengths, x.q_lengths)
+        tf = flops / (ms * 1e-3) / 1e12
+        row = {"workload": w.name, "value": tf, "unit": "TFLOP/s", "ms_per_launch": ms,
+               "flops_per_launch": flops, "launches": steps, "l2": "flushed before each launch",
+               "roofline": {"bound": "tensor", "achieved": tf, "peak": peak, "unit": "TFLOP/s",
+                            "frac": tf / peak, "traffic": None,
+                            "kernel": f"attn_fwd_kernel<{w.D}>"}}
+        if x.k_lengths is not None and key == "window":
+            row["lengths"] = x.k_lengths.tolist()
+        if key == "tiny":
+            row["latency_us"] = 1e3 * ms
+        if orc is not None and key != "tiny":
+            stride = 256 if key == "window" else 64
+            f, dt, nrows = oracle_sample_prefill(orc, w, x, stride)
+            row["cpu_baseline"] = {
+                "value": f / dt / 1e12, "unit": "TFLOP/s", "cores": orc.num_threads(),
+                "kind": "oracle",
+                "sample": f"query rows i % {stride} == 0 ({nrows} rows) of every (batch, head): "
+                          f"{f:.3e} algorithmic FLOP in {dt:.2f} s"}
+        out[key] = row
+        del Q, K, V, O, LSE
         torch.cuda.empty_cache()
     return out
 
@@ -625,6 +706,9 @@ def main(argv=None):
                     help="skip the flex_attention! measurements (reported apart from the step)")
     ap.add_argument("--no-bwd", action="store_true",
                     help="skip the backward measurement (reported apart from the step)")
+    ap.add_argument("--no-configs", action="store_true",
+                    help="skip the window / image / tiny prefill rows (reported apart from "
+                         "the step)")
     ap.add_argument("--no-paged", action="store_true",
                     help="skip the paged-KV decode measurement (reported apart from the step)")
     ap.add_argument("--only", choices=["prefill", "decode", "flex", "paged", "bwd"], default=None,
@@ -737,6 +821,10 @@ def main(argv=None):
         line["e2e"] = e2e
     if world == 1 and not args.no_cpu_baseline:
         line["cpu_baseline"] = cpu_baseline(step.host_prefill, step.dQ_host, step.lengths_host)
+    if not args.no_configs and step.do_prefill:
+        line["prefill_configs"] = time_prefill_configs(
+            dev, min(K, 50), args.warmup, peaks["bf16_tflops"],
+            world == 1 and not args.no_cpu_baseline)
     if not args.no_flex:
         line["flex"] = time_flex(dev, min(K, 50), args.warmup, peaks["bf16_tflops"])
     if not args.no_flex:
