@@ -14,10 +14,14 @@ import os
 import torch
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
-LIBRARY = os.path.join(_HERE, "libgqa_attn.so")
+# GQA_ATTN_DEBUG=1 selects the checked build (every TMA coordinate and global
+# index range-checked in the kernels; built with `... build --debug`).
+CHECKED = os.environ.get("GQA_ATTN_DEBUG", "0") == "1"
+LIBRARY = os.path.join(_HERE, "libgqa_attn_debug.so" if CHECKED else "libgqa_attn.so")
 
 if not os.path.exists(LIBRARY):
-    raise ImportError(f"{LIBRARY} is not built; run `python -m gqa_attention_flash_b200.build`")
+    raise ImportError(f"{LIBRARY} is not built; run `python -m gqa_attention_flash_b200.build"
+                      f"{' --debug' if CHECKED else ''}`")
 
 lib = ctypes.CDLL(LIBRARY)
 

@@ -292,8 +292,12 @@ __global__ void __launch_bounds__(kThreadsTc, 1)
                 prefetch_tensormap(&tmK);
                 prefetch_tensormap(&tmV);
                 prefetch_tensormap(&tmdO);
-                mbar_arrive_expect_tx(bar(C::BAR_RES), 2 * C::TILE);
-                for (int c = 0; c < C::NBOX; ++c) {
+                // checked build: the resident K / V tile lies inside the tensors
+                if (in_range(box_ok(0, kv0, b * p.Hkv + hkv, D, p.Sk, (long long)p.B * p.Hkv, TB) &&
+                                 kv0 >= 0 && kv0 < p.Sk,
+                             p.status, abort_flag))
+                    mbar_arrive_expect_tx(bar(C::BAR_RES), 2 * C::TILE);
+                for (int c = 0; c < C::NBOX && !*abort_flag; ++c) {
                     tma_load_3d(sbase + C::OFF_R0 + c * C::BOX, &tmK, bar(C::BAR_RES), c * 64, kv0,
                                 b * p.Hkv + hkv);
                     tma_load_3d(sbase + C::OFF_R1 + c * C::BOX, &tmV, bar(C::BAR_RES), c * 64, kv0,
@@ -305,6 +309,11 @@ __global__ void __launch_bounds__(kThreadsTc, 1)
                 const int hq = hkv * p.group + it / n_qt;
                 const int q0 = (qt_lo + it % n_qt) * TB;
                 const long long qrow = (long long)(b * p.Hq + hq) * p.Sq;
+                // checked build: this item's Q / dO tiles and LSE / delta rows exist
+                if (!in_range(hq < p.Hq && box_ok(0, q0, b * p.Hq + hq, D, p.Sq, (long long)p.B * p.Hq,
+                                                  TB) && q0 >= 0 && q0 < p.Sq,
+                              p.status, abort_flag))
+                    break;
                 // the tile's -LSE (log2 units) and -delta, loaded before the slot is free
                 float lr[TB / 32], dr[TB / 32];
 #pragma unroll
@@ -576,8 +585,12 @@ __global__ void __launch_bounds__(kThreadsTc, 1)
             prefetch_tensormap(&tmK);
             prefetch_tensormap(&tmV);
             prefetch_tensormap(&tmdO);
-            mbar_arrive_expect_tx(bar(C::BAR_RES), 2 * C::TILE);
-            for (int c = 0; c < C::NBOX; ++c) {
+            // checked build: the resident Q / dO tile lies inside the tensors
+            if (in_range(box_ok(0, q0, b * p.Hq + hq, D, p.Sq, (long long)p.B * p.Hq, TB) && q0 >= 0 &&
+                             q0 < p.Sq,
+                         p.status, abort_flag))
+                mbar_arrive_expect_tx(bar(C::BAR_RES), 2 * C::TILE);
+            for (int c = 0; c < C::NBOX && !*abort_flag; ++c) {
                 tma_load_3d(sbase + C::OFF_Q + c * C::BOX, &tmQ, bar(C::BAR_RES), c * 64, q0,
                             b * p.Hq + hq);
                 tma_load_3d(sbase + C::OFF_DO + c * C::BOX, &tmdO, bar(C::BAR_RES), c * 64, q0,
@@ -586,6 +599,10 @@ __global__ void __launch_bounds__(kThreadsTc, 1)
             for (int g = 0; g < n_kt; ++g) {
                 const int kv0 = (lo + g) * TB;
                 const int ks = g % C::NK, ku = g / C::NK, vs = g % C::NV, vu = g / C::NV;
+                if (!in_range(box_ok(0, kv0, b * p.Hkv + hkv, D, p.Sk, (long long)p.B * p.Hkv, TB) &&
+                                  kv0 >= 0 && kv0 < p.Sk,
+                              p.status, abort_flag))
+                    break;
                 if (ku > 0 && !mbar_wait(bar(C::BAR_EMPTYK + ks), (ku - 1) & 1, abort_flag,
                                          p.wait_limit_ns, p.status))
                     break;

@@ -112,9 +112,14 @@ __global__ void __launch_bounds__(kDecThreads)
 
     float *ws_base = p.ws + ((long long)(b * p.Hq + h0) * p.n_splits + split) * C::WS_STRIDE;
     const long long ws_head = (long long)p.n_splits * C::WS_STRIDE;
+    // checked build: the workspace entries of this CTA's G heads lie inside it
+    const long long ws_end = (long long)p.B * p.Hq * p.n_splits * C::WS_STRIDE;
+    const bool ws_ok = in_range(
+        ((long long)(b * p.Hq + h0 + G - 1) * p.n_splits + split) * C::WS_STRIDE + D < ws_end,
+        p.status, nullptr);
 
     if (k0 >= k1) {  // empty slice: weight zero in the combine
-        for (int h = threadIdx.x; h < G; h += blockDim.x) ws_base[h * ws_head + D] = neg_inf();
+        for (int h = threadIdx.x; h < G && ws_ok; h += blockDim.x) ws_base[h * ws_head + D] = neg_inf();
         return;
     }
     const int t_begin = k0 / TN;
@@ -143,6 +148,11 @@ __global__ void __launch_bounds__(kDecThreads)
                     break;
                 const int row = (t_begin + it) * TN;
                 if constexpr (!kPaged) {
+                    if (!in_range(box_ok(0, row, b * p.Hkv + hkv, D, p.S_cap, (long long)p.B * p.Hkv,
+                                         TN) &&
+                                      row >= 0 && row < p.S_cap,
+                                  p.status, abort_flag))
+                        break;
                     mbar_arrive_expect_tx(full(st), 2 * C::TILE);
                     for (int c = 0; c < C::NBOX; ++c) {
                         tma_load_3d(sbase + C::OFF_K + st * C::TILE + c * C::BOX, &tmK, full(st),
@@ -165,6 +175,9 @@ __global__ void __launch_bounds__(kDecThreads)
                         if (blk < 0 || blk >= p.num_blocks) record_status(p.status, ATTN_ERR_DEVICE_BOUNDS);
                         // an out-of-range block reads as zeros (outside the tensor map)
                         const int prow = blk * (1 << p.block_shift) + (j & ((1 << p.block_shift) - 1));
+                        // checked build: the chunk stays inside its tile of the ring (an
+                        // out-of-range block is the documented zero-filled case)
+                        if (!in_range(k * br + br <= TN && hkv < p.Hkv, p.status, abort_flag)) break;
                         for (int c = 0; c < C::NBOX; ++c) {
                             const uint32_t off = st * C::TILE + c * C::BOX + k * br * 128;
                             tma_load_3d(sbase + C::OFF_K + off, &tmK, full(st), c * 64, hkv, prow);
@@ -324,7 +337,7 @@ __global__ void __launch_bounds__(kDecThreads)
             ml[warp * kMaxGroup + g + 8] = l_run[1];
         }
         asm volatile("bar.sync 1, %0;" ::"n"(32 * kConsumers) : "memory");
-        if (ok && !*abort_flag) {
+        if (ok && !*abort_flag && ws_ok) {
             for (int idx = threadIdx.x; idx < G * D; idx += 32 * kConsumers) {
                 const int h = idx / D, d = idx % D;
                 float M = neg_inf();
@@ -345,7 +358,8 @@ __global__ void __launch_bounds__(kDecThreads)
             // A bounded wait ran out: the slice weighs nothing in the combine, so
             // whatever the workspace held before (another call's partials) never
             // reaches O.
-            for (int h = threadIdx.x; h < G; h += 32 * kConsumers) ws_base[h * ws_head + D] = neg_inf();
+            for (int h = threadIdx.x; h < G && ws_ok; h += 32 * kConsumers)
+                ws_base[h * ws_head + D] = neg_inf();
         }
     }
     if (*abort_flag) drain_delay(2000000);

@@ -19,6 +19,39 @@ __device__ __forceinline__ void record_status(int *status, int code) {
     if (status) atomicCAS(status, 0, code);
 }
 
+// Checked build (compiled with GQA_ATTN_DEBUG, library libgqa_attn_debug.so):
+// every TMA coordinate and every global index a kernel is about to use is
+// range-checked first.  A failed check records ATTN_ERR_DEVICE_BOUNDS, raises the
+// block's abort flag (so every role heads for its exit path, as after a bounded
+// wait that ran out) and the access is skipped; nothing traps.  In the normal
+// build in_range() is the constant true and the checks compile to nothing.
+#ifdef GQA_ATTN_DEBUG
+constexpr bool kChecked = true;
+#else
+constexpr bool kChecked = false;
+#endif
+
+__device__ __forceinline__ bool in_range(bool ok, int *status, volatile int *abort_flag) {
+    if constexpr (kChecked) {
+        if (!ok) {
+            record_status(status, ATTN_ERR_DEVICE_BOUNDS);
+            if (abort_flag) *abort_flag = 1;
+        }
+        return ok;
+    }
+    return true;
+}
+
+// A TMA box load (or store) of `box_rows` x 64 bf16 at (x, y, z) into a
+// (X, Y, Z) tensor: x is a multiple of 64 (16-byte aligned) inside [0, X), z
+// inside [0, Z) and the box starts at most one box above or below the rows
+// (rows outside read as zeros; stores are clipped).
+__device__ __forceinline__ bool box_ok(int x, int y, int z, int X, long long Y, long long Z,
+                                       int box_rows) {
+    return x >= 0 && (x & 63) == 0 && x + 64 <= X && y > -box_rows && y < Y + box_rows && z >= 0 &&
+           z < Z;
+}
+
 __device__ __forceinline__ uint32_t smem_u32(const void *p) {
     return static_cast<uint32_t>(__cvta_generic_to_shared(p));
 }
@@ -123,6 +156,39 @@ __device__ __forceinline__ void tma_load_3d(uint32_t dst, const void *tmap, uint
         " [%0], [%1, {%3, %4, %5}], [%2];" ::"r"(dst),
         "l"(reinterpret_cast<uint64_t>(tmap)), "r"(bar), "r"(x), "r"(y), "r"(z)
         : "memory");
+}
+
+// ---------------------------------------------------------------------------------
+// Cluster launch control (sm_100): a running CTA takes over the work of a CTA of
+// the same grid that has not been launched yet, so a grid of one CTA per work
+// item runs as one persistent CTA per SM while keeping the launch order.
+// ---------------------------------------------------------------------------------
+// Request the cancellation of one not-yet-launched CTA.  The 16-byte response
+// lands in shared memory at `resp` (16-byte aligned) and completes `bar` as 16
+// transaction bytes (the caller arms it with mbar_arrive_expect_tx(bar, 16)).
+// After a response that cancelled nothing, no further request may be made.
+__device__ __forceinline__ void clc_try_cancel(uint32_t resp, uint32_t bar) {
+    asm volatile(
+        "clusterlaunchcontrol.try_cancel.async.shared::cta.mbarrier::complete_tx::bytes.b128"
+        " [%0], [%1];" ::"r"(resp),
+        "r"(bar)
+        : "memory");
+}
+
+// Decode a response: the x index of the cancelled CTA, or -1 when none was
+// cancelled (the grid has no CTA left to launch).
+__device__ __forceinline__ int clc_cancelled_x(uint32_t resp) {
+    uint32_t x = 0xffffffffu, ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t.reg .b128 r;\n\t"
+        "ld.shared.b128 r, [%2];\n\t"
+        "clusterlaunchcontrol.query_cancel.is_canceled.pred.b128 p, r;\n\t"
+        "selp.u32 %1, 1, 0, p;\n\t"
+        "@p clusterlaunchcontrol.query_cancel.get_first_ctaid::x.b32.b128 %0, r;\n\t}"
+        : "+r"(x), "=r"(ok)
+        : "r"(resp)
+        : "memory");
+    return ok ? static_cast<int>(x) : -1;
 }
 
 // ---------------------------------------------------------------------------------

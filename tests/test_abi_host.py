@@ -40,6 +40,14 @@ def test_library_exports_every_declared_symbol(binding):
         assert isinstance(getattr(binding.lib, name), ctypes._CFuncPtr)
 
 
+def test_checked_library_exports_every_declared_symbol():
+    """The range-checked build (GQA_ATTN_DEBUG) exports the same C ABI."""
+    from gqa_attention_flash_b200 import build
+    lib = ctypes.CDLL(build.build(debug=True))
+    for name in declared_functions():
+        assert hasattr(lib, name), name
+
+
 def test_status_strings(binding):
     for code, name in binding.STATUS.items():
         assert binding.status_string(code).startswith(name)
