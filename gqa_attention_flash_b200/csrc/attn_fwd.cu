@@ -379,6 +379,11 @@ __global__ void __launch_bounds__(kThreads, 1)
             prefetch_tensormap(&tmQ);
             prefetch_tensormap(&tmK);
             prefetch_tensormap(&tmV);
+            // L2 policies: each Q tile is read once (evict first); the K / V tiles of a
+            // KV head serve every query tile and query head of its group (evict last).
+            // DRAM traffic of the LLM workload: 393 -> 335 MB per launch (322 MB of
+            // inputs and outputs), at the same speed.
+            const uint64_t pol_q = l2_policy_evict_first(), pol_kv = l2_policy_evict_last();
             bool more = !kList;  // launch-control requests still allowed
             bool ok = true;
             uint32_t qi = 0;     // Q tiles loaded so far: slot qi % NQ, use qi / NQ
@@ -403,9 +408,9 @@ __global__ void __launch_bounds__(kThreads, 1)
                         return false;
                     mbar_arrive_expect_tx(bar(C::BAR_QFULL + slot), C::Q_BYTES);
                     for (int c = 0; c < C::NBOX; ++c)
-                        tma_load_3d(sbase + C::OFF_Q + slot * C::Q_BYTES + c * C::BOX, &tmQ,
-                                         bar(C::BAR_QFULL + slot), c * 64,
-                                         (it.pair * kTiles + t) * BM, it.b * p.Hq + it.hq);
+                        tma_load_3d_hint(sbase + C::OFF_Q + slot * C::Q_BYTES + c * C::BOX, &tmQ,
+                                         bar(C::BAR_QFULL + slot), c * 64, (it.pair * kTiles + t) * BM,
+                                         it.b * p.Hq + it.hq, pol_q);
                     ++qi;
                     return true;
                 };
@@ -425,14 +430,14 @@ __global__ void __launch_bounds__(kThreads, 1)
                         return false;
                     mbar_arrive_expect_tx(bar(C::BAR_KFULL + st), C::KV_BYTES);
                     for (int c = 0; c < C::NBOX; ++c)
-                        tma_load_3d(sbase + C::OFF_K + st * C::KV_BYTES + c * C::BOX, &tmK,
+                        tma_load_3d_hint(sbase + C::OFF_K + st * C::KV_BYTES + c * C::BOX, &tmK,
                                          bar(C::BAR_KFULL + st), c * 64, kv_row,
-                                         it.b * p.Hkv + it.hkv);
+                                         it.b * p.Hkv + it.hkv, pol_kv);
                     mbar_arrive_expect_tx(bar(C::BAR_VFULL + st), C::KV_BYTES);
                     for (int c = 0; c < C::NBOX; ++c)
-                        tma_load_3d(sbase + C::OFF_V + st * C::KV_BYTES + c * C::BOX, &tmV,
+                        tma_load_3d_hint(sbase + C::OFF_V + st * C::KV_BYTES + c * C::BOX, &tmV,
                                          bar(C::BAR_VFULL + st), c * 64, kv_row,
-                                         it.b * p.Hkv + it.hkv);
+                                         it.b * p.Hkv + it.hkv, pol_kv);
                     ++gi;
                     return true;
                 };
