@@ -51,24 +51,37 @@ __global__ void __launch_bounds__(128)
     for (int i = tid; i < n * D / 8; i += blockDim.x)  // 16-byte loads (rows are 16B-aligned)
         reinterpret_cast<uint4 *>(kblk)[i] = reinterpret_cast<const uint4 *>(Kb)[i];
     __syncthreads();
-    if (tid < D) {
-        float acc = 0.f;
-#pragma unroll 8
-        for (int j = 0; j < n; ++j) acc += __bfloat162float(kblk[j * D + tid]);
-        c[tid] = acc / static_cast<float>(n);
+    if (tid < D) {  // column sums on four independent chains
+        float acc[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll 4
+        for (int j = 0; j < n; ++j) acc[j & 3] += __bfloat162float(kblk[j * D + tid]);
+        c[tid] = ((acc[0] + acc[1]) + (acc[2] + acc[3])) / static_cast<float>(n);
     }
     __syncthreads();
-    float rm = 0.f;
-    for (int j = warp; j < n; j += 4) {
-        float ss = 0.f;
-        for (int d = lane; d < D; d += 32) {
-            const float e = __bfloat162float(kblk[j * D + d]) - c[d];
-            ss = fmaf(e, e, ss);
-        }
+    // |k - c|^2 of the warp's 16 rows (rows warp, warp + 4, ...), each lane summing
+    // its D / 32 columns; the 16 row sums are independent, so their loads and the
+    // cross-lane reductions overlap instead of running row after row
+    constexpr int kRowsPerWarp = kBlk / 4;
+    float ss[kRowsPerWarp];
 #pragma unroll
-        for (int o = 16; o > 0; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
-        rm = fmaxf(rm, sqrtf(ss));
+    for (int i = 0; i < kRowsPerWarp; ++i) {
+        const int j = warp + 4 * i;
+        ss[i] = 0.f;
+        if (j < n) {
+#pragma unroll
+            for (int d = lane; d < D; d += 32) {
+                const float e = __bfloat162float(kblk[j * D + d]) - c[d];
+                ss[i] = fmaf(e, e, ss[i]);
+            }
+        }
     }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1)
+#pragma unroll
+        for (int i = 0; i < kRowsPerWarp; ++i) ss[i] += __shfl_xor_sync(0xffffffffu, ss[i], o);
+    float rm = 0.f;
+#pragma unroll
+    for (int i = 0; i < kRowsPerWarp; ++i) rm = fmaxf(rm, sqrtf(ss[i]));  // rows past n hold 0
     if (lane == 0) rmax_w[warp] = rm;
     const long long row = (long long)(b * Hkv + hkv) * nkb + kb;
     if (tid < D) {  // the centroid as bf16 high part + bf16 remainder
@@ -165,6 +178,7 @@ __global__ void __launch_bounds__(128) rbs_scores_kernel(const ScoreParams p) {
     float *sb = red + 4 * 64 * 4;         // [nkb] base scores of this row
     float *sr = sb + p.nkb;               // [nkb] rescue scores
     __shared__ float red2[2][4];
+    __shared__ float rb_s[64];  // radius * beta of the key blocks of the current group
     const int qb = blockIdx.x, hq = blockIdx.y, b = blockIdx.z;
     const int hkv = hq / p.group;
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -186,6 +200,7 @@ __global__ void __launch_bounds__(128) rbs_scores_kernel(const ScoreParams p) {
         const int nk = min(64, p.nkb - g0);
         stage64<D>(ch_tile, p.cent_hi + (hrow + g0) * D, nk);
         stage64<D>(cl_tile, p.cent_lo + (hrow + g0) * D, nk);
+        if (tid < 64) rb_s[tid] = tid < nk ? p.rad[hrow + g0 + tid] * p.beta[hrow + g0 + tid] : 0.f;
         __syncthreads();
         if (g0 == 0) {
             float q0 = 0.f, q1 = 0.f;  // partial |q|^2 of rows r, r + 8
@@ -232,7 +247,7 @@ __global__ void __launch_bounds__(128) rbs_scores_kernel(const ScoreParams p) {
             for (int e = 0; e < 2; ++e) {
                 const int col = 8 * j + 2 * t + e;  // key block g0 + col
                 const int kb = g0 + col;
-                const float rb = kb < p.nkb ? p.rad[hrow + kb] * p.beta[hrow + kb] : 0.f;
+                const float rb = rb_s[col];
                 const float s0 = acc[j][e], s1 = acc[j][2 + e];
                 const float b0 = v0 ? s0 * inv_sqrt_d : ninf, b1 = v1 ? s1 * inv_sqrt_d : ninf;
                 const float x0 = v0 ? fmaf(qn0, rb, s0) * inv_sqrt_d : ninf;
