@@ -252,51 +252,99 @@ def time_device(step, steps, warmup, barrier):
 
 
 def time_e2e(step, steps, warmup):
-    """Same step through the public API with pinned HOST inputs and outputs: every
-    step copies the prefill's Q/K/V/k_lengths and the decode's Q/lengths host->
-    device and reads O/LSE and the decode O back.  The 8.6 GB KV cache is decode
-    state and stays resident."""
+    """Same work through the public API with pinned HOST inputs and outputs: every
+    step copies the prefill's Q/K/V/k_lengths (or the decode's Q/lengths) host->
+    device and reads O/LSE (or the decode O) back.  The 8.6 GB KV cache is decode
+    state and stays resident.
+
+    Steps are pipelined the way a serving loop would run them: one stream copies
+    step i+1's inputs in, one runs step i's kernels, one copies step i-1's outputs
+    out, on two sets of device buffers (PCIe is full duplex, so the two copy
+    directions overlap each other and the kernels).  Each of the two halves is
+    timed from the first copy-in to the last copy-out over `steps` steps."""
+    from gqa_attention_flash_b200 import binding
+    dev = step.dev
     x = step.host_prefill
     hQ, hK, hV = x.Q.pin_memory(), x.K.pin_memory(), x.V.pin_memory()
     hkl = x.k_lengths.pin_memory()
     hdQ, hlen = step.dQ_host.pin_memory(), step.lengths_host.pin_memory()
-    oO = torch.empty(step.O.shape, dtype=step.O.dtype).pin_memory()
-    oL = torch.empty(step.LSE.shape, dtype=step.LSE.dtype).pin_memory()
-    odO = torch.empty(step.dO.shape, dtype=step.dO.dtype).pin_memory()
-    s = torch.cuda.current_stream()
     h2d = sum(t.numel() * t.element_size() for t in (hQ, hK, hV, hkl, hdQ, hlen))
-    d2h = sum(t.numel() * t.element_size() for t in (oO, oL, odO))
+    d2h = (step.O.numel() * step.O.element_size() + step.LSE.numel() * step.LSE.element_size()
+           + step.dO.numel() * step.dO.element_size())
+    w = step.pw
+    s_in, s_cmp, s_out = torch.cuda.Stream(dev), torch.cuda.Stream(dev), torch.cuda.Stream(dev)
 
-    def one():
-        step.Q.copy_(hQ, non_blocking=True)
-        step.K.copy_(hK, non_blocking=True)
-        step.V.copy_(hV, non_blocking=True)
-        step.kl.copy_(hkl, non_blocking=True)
-        step.prefill()
-        oO.copy_(step.O, non_blocking=True)
-        oL.copy_(step.LSE, non_blocking=True)
+    # prefill buffers: [device inputs, device outputs, host outputs] x 2
+    pb = [dict(Q=torch.empty_like(step.Q), K=torch.empty_like(step.K), V=torch.empty_like(step.V),
+               kl=torch.empty_like(step.kl), O=torch.empty_like(step.O),
+               L=torch.empty_like(step.LSE),
+               hO=torch.empty(step.O.shape, dtype=step.O.dtype).pin_memory(),
+               hL=torch.empty(step.LSE.shape, dtype=step.LSE.dtype).pin_memory())
+          for _ in range(2)]
+    db = [dict(Q=torch.empty_like(step.dQ), n=torch.empty_like(step.lengths),
+               O=torch.empty_like(step.dO),
+               hO=torch.empty(step.dO.shape, dtype=step.dO.dtype).pin_memory())
+          for _ in range(2)]
 
-    def two():
-        step.dQ.copy_(hdQ, non_blocking=True)
-        step.lengths.copy_(hlen, non_blocking=True)
-        step.decode()
-        odO.copy_(step.dO, non_blocking=True)
+    def pre_in(b):
+        b["Q"].copy_(hQ, non_blocking=True)
+        b["K"].copy_(hK, non_blocking=True)
+        b["V"].copy_(hV, non_blocking=True)
+        b["kl"].copy_(hkl, non_blocking=True)
 
-    for _ in range(warmup):
-        one()
-        two()
-    torch.cuda.synchronize()
-    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True),
-           torch.cuda.Event(enable_timing=True)) for _ in range(steps)]
-    for e0, e1, e2 in ev:
-        e0.record(s)
-        one()
-        e1.record(s)
-        two()
-        e2.record(s)
-    torch.cuda.synchronize()
-    p_ms = sum(e0.elapsed_time(e1) for e0, e1, _ in ev)
-    d_ms = sum(e1.elapsed_time(e2) for _, e1, e2 in ev)
+    def pre_run(b):
+        binding.attn_fwd(b["O"], b["Q"], b["K"], b["V"], b["L"], w.scale, w.causal, w.window,
+                         w.input_pos, b["kl"], stream=s_cmp)
+
+    def pre_out(b):
+        b["hO"].copy_(b["O"], non_blocking=True)
+        b["hL"].copy_(b["L"], non_blocking=True)
+
+    def dec_in(b):
+        b["Q"].copy_(hdQ, non_blocking=True)
+        b["n"].copy_(hlen, non_blocking=True)
+
+    def dec_run(b):
+        binding.attn_decode(b["O"], b["Q"], step.Kc, step.Vc, b["n"], step.dw.n_splits,
+                            stream=s_cmp)
+
+    def dec_out(b):
+        b["hO"].copy_(b["O"], non_blocking=True)
+
+    def pipeline(bufs, cin, run, cout, n):
+        torch.cuda.synchronize()
+        start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        ev_in = [torch.cuda.Event() for _ in range(n)]
+        ev_cmp = [torch.cuda.Event() for _ in range(n)]
+        ev_out = [torch.cuda.Event() for _ in range(n)]
+        start.record(s_in)
+        for i in range(n):
+            b = bufs[i % 2]
+            if i >= 2:
+                s_in.wait_event(ev_cmp[i - 2])   # step i-2 no longer reads these inputs
+            with torch.cuda.stream(s_in):
+                cin(b)
+            ev_in[i].record(s_in)
+            s_cmp.wait_event(ev_in[i])
+            if i >= 2:
+                s_cmp.wait_event(ev_out[i - 2])  # step i-2's outputs are on the host
+            run(b)
+            ev_cmp[i].record(s_cmp)
+            s_out.wait_event(ev_cmp[i])
+            with torch.cuda.stream(s_out):
+                cout(b)
+            ev_out[i].record(s_out)
+        end.record(s_out)
+        torch.cuda.synchronize()
+        return start.elapsed_time(end)
+
+    pipeline(pb, pre_in, pre_run, pre_out, warmup)
+    p_ms = pipeline(pb, pre_in, pre_run, pre_out, steps)
+    pipeline(db, dec_in, dec_run, dec_out, warmup)
+    d_ms = pipeline(db, dec_in, dec_run, dec_out, steps)
+    st = binding.last_device_status(s_cmp)
+    if st != 0:
+        raise RuntimeError(f"e2e device status: {binding.status_string(st)}")
     return p_ms, d_ms, h2d, d2h
 
 
@@ -777,8 +825,9 @@ def main(argv=None):
         e2e = {"value": e["flops"] / (e["p_ms"] * 1e-3) / 1e12, "unit": "TFLOP/s",
                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                "decode": {"value": e["bytes"] / (e["d_ms"] * 1e-3) / 1e9, "unit": "GB/s"},
-               "note": "pinned host Q/K/V/lengths -> device and O/LSE -> host every step; "
-                       "the decode KV cache is resident state"}
+               "note": "pinned host Q/K/V/lengths -> device and O/LSE -> host every step, "
+                       "steps pipelined over three streams (copy in / kernels / copy out) on "
+                       "two buffer sets; the decode KV cache is resident state"}
     if world > 1:
         barrier()
     if rank != 0:
