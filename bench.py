@@ -537,9 +537,10 @@ def time_prefill_configs(dev, steps, warmup, peak, with_cpu):
 def time_block_sparse(dev, steps, warmup, peak):
     """Block-sparse prefill row on the block-structured image workload: RBS block scores + mask
     (attn_rbs_block_mask), then attention over the kept 64x64 blocks (attn_fwd_flex,
-    per-head masks); CUDA events per launch.  TFLOP/s counts the kept pairs; the
-    dense attention of the same inputs is timed beside it."""
+    per-head masks); CUDA events per launch, L2 flushed before each.  TFLOP/s counts
+    the kept pairs; the dense attention of the same inputs is timed beside it."""
     from gqa_attention_flash_b200 import binding
+    flush = L2Flush(dev)
     w = W.BLOCK_SPARSE
     x = W.make_prefill(w)
     Q, K, V = x.Q.to(dev), x.K.to(dev), x.V.to(dev)
@@ -563,6 +564,7 @@ def time_block_sparse(dev, steps, warmup, peak):
         ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
               for _ in range(steps)]
         for e0, e1 in ev:
+            flush()
             e0.record()
             fn()
             e1.record()
@@ -582,8 +584,9 @@ def time_block_sparse(dev, steps, warmup, peak):
             "unit": "TFLOP/s (kept blocks)", "density": kept / total,
             "estimator_ms": t_est, "sparse_attention_ms": t_sparse, "dense_attention_ms": t_dense,
             "speedup_vs_dense": t_dense / (t_est + t_sparse), "launches": steps,
+            "l2": "flushed before each launch",
             "roofline": {"bound": "tensor", "achieved": tf, "peak": peak, "unit": "TFLOP/s",
-                         "frac": tf / peak, "kernel": "attn_fwd_kernel<128, flex, block list>"}}
+                         "frac": tf / peak, "kernel": "attn_fwd_bsparse_kernel<128>"}}
 
 
 def time_backward(step, steps, warmup, peak):

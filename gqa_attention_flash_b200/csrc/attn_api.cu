@@ -42,7 +42,7 @@ std::mutex g_setup_mutex;
 std::set<std::pair<int, const void *>> g_setup_done;
 }  // namespace
 
-cudaError_t kernel_setup(const void *func, int smem_bytes, int required_regs) {
+cudaError_t kernel_setup(const void *func, int smem_bytes, int required_regs, bool max_smem_carveout) {
     int dev = -1;
     cudaError_t e = cudaGetDevice(&dev);
     if (e != cudaSuccess) return e;
@@ -55,6 +55,10 @@ cudaError_t kernel_setup(const void *func, int smem_bytes, int required_regs) {
     }
     if ((e = cudaFuncSetAttribute(func, cudaFuncAttributeMaxDynamicSharedMemorySize, smem_bytes)) !=
         cudaSuccess)
+        return e;
+    if (max_smem_carveout &&
+        (e = cudaFuncSetAttribute(func, cudaFuncAttributePreferredSharedMemoryCarveout,
+                                  cudaSharedmemCarveoutMaxShared)) != cudaSuccess)
         return e;
     g_setup_done.insert({dev, func});
     return cudaSuccess;
@@ -301,6 +305,7 @@ attn_status_t attn_fwd_flex(void *O, const void *Q, const void *K, const void *V
         a.doc_q = nullptr;
         a.block_mask = nullptr;
     }
+    if (gqa::bsparse_eligible(a)) return gqa::launch_fwd_bsparse(a, static_cast<cudaStream_t>(stream));
     return launch_fwd(a, static_cast<cudaStream_t>(stream));
 }
 

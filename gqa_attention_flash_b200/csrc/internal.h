@@ -41,6 +41,14 @@ struct FwdArgs {
 // of visited tiles lives in shared memory).
 constexpr int kFlexMaxKvTiles = 1024;
 
+// Block-sparse prefill kernel (BlockMask alone, no score mod, no DocumentMask,
+// not causal, no lengths): longest key sequence it takes, in 64-key blocks (its
+// per-CTA list of visited blocks lives in shared memory).  Other flex calls, and
+// longer sequences, run on the flex kernel's list path.
+constexpr int kBsparseMaxKvBlocks = 1024;
+bool bsparse_eligible(const FwdArgs &a);
+attn_status_t launch_fwd_bsparse(const FwdArgs &a, cudaStream_t stream);
+
 struct DecodeArgs {
     void *O;
     const void *Q, *K, *V;
@@ -92,9 +100,12 @@ attn_status_t launch_decode(const DecodeArgs &a, cudaStream_t stream);
 attn_status_t launch_wait_probe(int limit_us, cudaStream_t stream);
 
 // Once per (device, kernel), thread-safe: check that the kernel was built with
-// `required_regs` registers per thread (skipped when negative) and raise its
-// dynamic shared-memory limit to `smem_bytes` on the current device.
-cudaError_t kernel_setup(const void *func, int smem_bytes, int required_regs = -1);
+// `required_regs` registers per thread (skipped when negative), raise its
+// dynamic shared-memory limit to `smem_bytes` on the current device and, with
+// max_smem_carveout, ask for the largest shared-memory carveout (kernels that
+// run several CTAs per SM, each with a large dynamic allocation).
+cudaError_t kernel_setup(const void *func, int smem_bytes, int required_regs = -1,
+                         bool max_smem_carveout = false);
 
 // Bounded-wait limit used by the attention kernels (nanoseconds of global time).
 constexpr uint64_t kWaitLimitNs = 2000000000ull;

@@ -4,7 +4,7 @@ In it every TMA coordinate and global index a kernel is about to use is checked
 first; a violation records ATTN_ERR_DEVICE_BOUNDS and the kernel gives up instead
 of touching memory outside its buffers.  This stands in for a memory checker: the
 small parity cases of every kernel family (prefill, flex, decode, paged decode,
-backward, RBS block scores and block-sparse attention, the bit-exact mask
+backward, RBS block scores, the block-sparse kernel, the bit-exact mask
 probes) run again in a child process that loads the checked library, and every
 one of them must pass with the device status word at ATTN_OK."""
 import os
@@ -38,6 +38,8 @@ SELECTION = [
     "test_gpu_bwd.py::test_backward_masked_rows_and_keys_are_zero",
     "test_gpu_rbs.py::test_rbs_scores_and_mask",
     "test_gpu_rbs.py::test_block_sparse_attention",
+    "test_gpu_bsparse.py::test_block_sparse_matches_oracle",
+    "test_gpu_bsparse.py::test_one_hot_probe_bit_exact",
 ]
 
 
