@@ -89,6 +89,20 @@ struct SpParams {
 
 __device__ __forceinline__ float sp_neg_inf() { return __int_as_float(0xff800000); }
 
+// Bring a 3-D tile of a tensor map into L2 ahead of its load (no shared memory,
+// no completion to wait for); x is a multiple of 64 elements.
+__device__ __forceinline__ void tma_prefetch_3d(const void *tmap, int x, int y, int z,
+                                                uint64_t policy) {
+    asm volatile(
+        "cp.async.bulk.prefetch.tensor.3d.L2.global.tile.L2::cache_hint [%0, {%1, %2, %3}], %4;" ::"l"(
+            reinterpret_cast<uint64_t>(tmap)),
+        "r"(x), "r"(y), "r"(z), "l"(policy)
+        : "memory");
+}
+
+// Key blocks whose K and V tiles are prefetched into L2 ahead of the block loaded.
+constexpr int kSpPrefetch = 4;
+
 template <int D>
 __global__ void __launch_bounds__(kSpThreads, 2)
     attn_fwd_bsparse_kernel(const __grid_constant__ CUtensorMap tmQ,
@@ -182,35 +196,61 @@ __global__ void __launch_bounds__(kSpThreads, 2)
                     tma_load_3d_hint(sbase + C::OFF_Q + c * C::Q_BOX, &tmQ, bar(C::BAR_QFULL), c * 64,
                                      qt * SP_BM, zq, pol_q);
             }
-            for (int j = 0; ok && j < n; ++j) {
+            // Checked build: the block lies inside K and V.
+            auto kv_row_of = [&](int j, int &row) -> bool {
+                row = (list[j] & 0x3FF) * SP_BN;
+                return in_range(box_ok(0, row, zk, D, p.Sk, (long long)p.B * p.Hkv, SP_BN) &&
+                                    row < p.Sk,
+                                p.status, abort_flag);
+            };
+            auto prefetch = [&](int j) {
+                int row;
+                if (j < n && kv_row_of(j, row)) {
+                    for (int c = 0; c < C::NBOX; ++c) {
+                        tma_prefetch_3d(&tmK, c * 64, row, zk, pol_kv);
+                        tma_prefetch_3d(&tmV, c * 64, row, zk, pol_kv);
+                    }
+                }
+            };
+            // K stage st is free once S of the block NS earlier is done; V stage st once
+            // P V of that block is done.
+            auto load_k = [&](int j) -> bool {
                 const int st = j % C::NS;
                 const uint32_t use = static_cast<uint32_t>(j / C::NS);
-                const int kv_row = (list[j] & 0x3FF) * SP_BN;
-                // checked build: the block lies inside K and V
-                if (!in_range(box_ok(0, kv_row, zk, D, p.Sk, (long long)p.B * p.Hkv, SP_BN) &&
-                                  kv_row < p.Sk,
-                              p.status, abort_flag)) {
-                    ok = false;
-                    break;
-                }
+                int row;
+                if (!kv_row_of(j, row)) return false;
                 if (use > 0 && !mbar_wait(bar(C::BAR_KEMPTY + st), (use - 1) & 1, abort_flag,
-                                          p.wait_limit_ns, p.status)) {
-                    ok = false;
-                    break;
-                }
+                                          p.wait_limit_ns, p.status))
+                    return false;
                 mbar_arrive_expect_tx(bar(C::BAR_KFULL + st), C::KV_BYTES);
                 for (int c = 0; c < C::NBOX; ++c)
                     tma_load_3d_hint(sbase + C::OFF_K + st * C::KV_BYTES + c * C::KV_BOX, &tmK,
-                                     bar(C::BAR_KFULL + st), c * 64, kv_row, zk, pol_kv);
+                                     bar(C::BAR_KFULL + st), c * 64, row, zk, pol_kv);
+                prefetch(j + kSpPrefetch);
+                return true;
+            };
+            auto load_v = [&](int j) -> bool {
+                const int st = j % C::NS;
+                const uint32_t use = static_cast<uint32_t>(j / C::NS);
+                int row;
+                if (!kv_row_of(j, row)) return false;
                 if (use > 0 && !mbar_wait(bar(C::BAR_VEMPTY + st), (use - 1) & 1, abort_flag,
-                                          p.wait_limit_ns, p.status)) {
-                    ok = false;
-                    break;
-                }
+                                          p.wait_limit_ns, p.status))
+                    return false;
                 mbar_arrive_expect_tx(bar(C::BAR_VFULL + st), C::KV_BYTES);
                 for (int c = 0; c < C::NBOX; ++c)
                     tma_load_3d_hint(sbase + C::OFF_V + st * C::KV_BYTES + c * C::KV_BOX, &tmV,
-                                     bar(C::BAR_VFULL + st), c * 64, kv_row, zk, pol_kv);
+                                     bar(C::BAR_VFULL + st), c * 64, row, zk, pol_kv);
+                return true;
+            };
+            for (int j = 1; ok && j < kSpPrefetch; ++j) prefetch(j);
+            // K runs one block ahead of V: S_{j+1} is needed before P_j V_j, and the
+            // stage K_{j+1} reuses is released (S_{j-1} done) before the one V_j
+            // reuses (P_{j-2} V_{j-2} done), so neither ring waits behind the other.
+            if (ok) ok = load_k(0);
+            for (int j = 0; ok && j < n; ++j) {
+                if (j + 1 < n) ok = load_k(j + 1);
+                if (ok) ok = load_v(j);
             }
         }
     } else if (warp == kSpWarpMma) {
@@ -297,13 +337,16 @@ __global__ void __launch_bounds__(kSpThreads, 2)
             }
             // online softmax in the exp2 domain; O is rescaled only when the row max
             // grows by more than 2^8
-            float mx0 = s[0], mx1 = s[1];
+            // row max: four independent chains of three-input maxima
+            float mx[4];
 #pragma unroll
-            for (int c = 2; c < SP_BN; c += 2) {
-                mx0 = fmaxf(mx0, s[c]);
-                mx1 = fmaxf(mx1, s[c + 1]);
+            for (int g = 0; g < 4; ++g) {
+                float a = fmax3(s[16 * g], s[16 * g + 1], s[16 * g + 2]);
+#pragma unroll
+                for (int c = 16 * g + 3; c < 16 * g + 15; c += 2) a = fmax3(a, s[c], s[c + 1]);
+                mx[g] = fmaxf(a, s[16 * g + 15]);
             }
-            const float m_new = fmaxf(mx0, mx1) * sl2;
+            const float m_new = fmax3(mx[0], mx[1], fmaxf(mx[2], mx[3])) * sl2;
             float alpha = 1.f;
             bool resc = false;
             if (m_new > m_used + 8.f) {
