@@ -36,6 +36,18 @@ namespace {
 
 constexpr int kBlk = 64;
 
+// 16-byte asynchronous copy global -> shared (cp.async); src_bytes 0 writes zeros.
+// Every copy a thread issues is in flight at once, so staging a tile costs one
+// memory round trip instead of one per loop iteration.
+__device__ __forceinline__ void cp_async16(uint32_t dst, const void *src, uint32_t src_bytes) {
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(dst), "l"(src), "r"(src_bytes)
+                 : "memory");
+}
+
+__device__ __forceinline__ void cp_async_wait_all() {
+    asm volatile("cp.async.wait_all;" ::: "memory");
+}
+
 template <int D>
 __global__ void __launch_bounds__(128)
     rbs_centroid_kernel(const __nv_bfloat16 *__restrict__ K, __nv_bfloat16 *__restrict__ cent_hi,
@@ -48,8 +60,9 @@ __global__ void __launch_bounds__(128)
     const int j0 = kb * kBlk, n = min(kBlk, Sk - j0);
     const __nv_bfloat16 *Kb = K + ((long long)(b * Hkv + hkv) * Sk + j0) * D;
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-    for (int i = tid; i < n * D / 8; i += blockDim.x)  // 16-byte loads (rows are 16B-aligned)
-        reinterpret_cast<uint4 *>(kblk)[i] = reinterpret_cast<const uint4 *>(Kb)[i];
+    for (int i = tid; i < n * D / 8; i += blockDim.x)  // 16-byte copies (rows are 16B-aligned)
+        cp_async16(smem_u32(kblk) + 16 * i, reinterpret_cast<const uint4 *>(Kb) + i, 16);
+    cp_async_wait_all();
     __syncthreads();
     if (tid < D) {  // column sums on four independent chains
         float acc[4] = {0.f, 0.f, 0.f, 0.f};
@@ -154,15 +167,17 @@ __device__ __forceinline__ uint32_t swz64(int row, int c) {
 }
 
 // Rows [0, n) of a row-major (., D) bf16 matrix into a swizzled 64-row tile
-// (rows n..63 zero), 16-byte loads spread over the block's threads.
+// (rows n..63 zero), 16-byte asynchronous copies spread over the block's
+// threads; the caller waits (cp_async_wait_all) and synchronises.
 template <int D>
 __device__ __forceinline__ void stage64(uint8_t *tile, const __nv_bfloat16 *src, int n) {
     constexpr int kChunks = D / 8;
+    const uint32_t t = smem_u32(tile);
     for (int i = threadIdx.x; i < 64 * kChunks; i += blockDim.x) {
         const int row = i / kChunks, c = i % kChunks;
-        uint4 v = make_uint4(0, 0, 0, 0);
-        if (row < n) v = __ldg(reinterpret_cast<const uint4 *>(src + (long long)row * D) + c);
-        *reinterpret_cast<uint4 *>(tile + swz64(row, c)) = v;
+        const bool in = row < n;
+        cp_async16(t + swz64(row, c),
+                   reinterpret_cast<const uint4 *>(src + (long long)(in ? row : 0) * D) + c, in ? 16u : 0u);
     }
 }
 
@@ -171,14 +186,15 @@ __global__ void __launch_bounds__(128) rbs_scores_kernel(const ScoreParams p) {
     extern __shared__ __align__(1024) uint8_t smraw[];
     constexpr int kKs = D / 16;           // k-steps of 16
     constexpr int kTile = 64 * D * 2;     // bytes of one staged 64-row tile
+    constexpr int kChunks = D / 8;        // 16-byte chunks per row
     uint8_t *q_tile = smraw;              // the query block
     uint8_t *ch_tile = smraw + kTile;     // centroids of a 64-block group: high parts
     uint8_t *cl_tile = smraw + 2 * kTile; // ... remainders
-    float *red = reinterpret_cast<float *>(smraw + 3 * kTile);  // [4][64][2 branches][max, sum]
-    float *sb = red + 4 * 64 * 4;         // [nkb] base scores of this row
+    float *sb = reinterpret_cast<float *>(smraw + 3 * kTile);  // [nkb] base scores of this row
     float *sr = sb + p.nkb;               // [nkb] rescue scores
     __shared__ float red2[2][4];
     __shared__ float rb_s[64];  // radius * beta of the key blocks of the current group
+    __shared__ float qn_s[64];  // |q| of the block's tokens
     const int qb = blockIdx.x, hq = blockIdx.y, b = blockIdx.z;
     const int hkv = hq / p.group;
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -186,114 +202,105 @@ __global__ void __launch_bounds__(128) rbs_scores_kernel(const ScoreParams p) {
     const int mi = lane >> 3, rr = lane & 7;  // ldmatrix: matrix of this lane's address, its row
     const int i0 = qb * kBlk, n_rows = min(kBlk, p.Sq - i0);
     const long long hrow = (long long)(b * p.Hkv + hkv) * p.nkb;
-    stage64<D>(q_tile, p.Q + ((long long)(b * p.Hq + hq) * p.Sq + i0) * D, n_rows);
-    // this warp's 16 token rows as m16n8k16 A fragments (rows r and r + 8)
-    const int r = warp * 16 + g;
-    const bool v0 = r < n_rows, v1 = r + 8 < n_rows;
-    const float inv_sqrt_d = rsqrtf(static_cast<float>(D));
+    // log2 units: scores scaled by log2(e) / sqrt(D), converted back at the end
+    const float k2 = rsqrtf(static_cast<float>(D)) * 1.4426950408889634f;
     const float ninf = __int_as_float(0xff800000);
     const uint32_t qs = smem_u32(q_tile), hs = smem_u32(ch_tile), ls = smem_u32(cl_tile);
-    uint32_t a[kKs][4];
-    float qn0 = 0.f, qn1 = 0.f;
-    // key blocks in groups of 64 = 8 n-tiles of 8
+    stage64<D>(q_tile, p.Q + ((long long)(b * p.Hq + hq) * p.Sq + i0) * D, n_rows);
+    // The product is taken transposed, S^T = C Q^T: warp w holds the 16 key blocks
+    // 16 w .. 16 w + 15 of a group (MMA rows) against all 64 tokens (MMA columns),
+    // so the log-sum-exp over the tokens of a key block runs over 16 values in each
+    // thread and then across the 4 lanes that share the row -- no cross-warp step.
+    float qn[8][2];  // |q| of this thread's tokens 8 j + 2 t + e
     for (int g0 = 0; g0 < p.nkb; g0 += 64) {
         const int nk = min(64, p.nkb - g0);
         stage64<D>(ch_tile, p.cent_hi + (hrow + g0) * D, nk);
         stage64<D>(cl_tile, p.cent_lo + (hrow + g0) * D, nk);
         if (tid < 64) rb_s[tid] = tid < nk ? p.rad[hrow + g0 + tid] * p.beta[hrow + g0 + tid] : 0.f;
+        cp_async_wait_all();  // (the query tile's copies too, on the first group)
         __syncthreads();
         if (g0 == 0) {
-            float q0 = 0.f, q1 = 0.f;  // partial |q|^2 of rows r, r + 8
+            // |q| of token tid / 2: each of two threads sums the squares of half the row
+            const int row = tid >> 1;
+            float q2 = 0.f;
 #pragma unroll
-            for (int kk = 0; kk < kKs; ++kk) {
-                ldmatrix_x4(qs + swz64(warp * 16 + (mi & 1) * 8 + rr, 2 * kk + (mi >> 1)), a[kk][0],
-                            a[kk][1], a[kk][2], a[kk][3]);
+            for (int c = (tid & 1) * (kChunks / 2); c < (tid & 1) * (kChunks / 2) + kChunks / 2; ++c) {
+                const uint4 v = *reinterpret_cast<const uint4 *>(q_tile + swz64(row, c));
+                const uint32_t w4[4] = {v.x, v.y, v.z, v.w};
 #pragma unroll
                 for (int e = 0; e < 4; ++e) {
-                    const __nv_bfloat162 h = *reinterpret_cast<const __nv_bfloat162 *>(&a[kk][e]);
+                    const __nv_bfloat162 h = *reinterpret_cast<const __nv_bfloat162 *>(&w4[e]);
                     const float x = __low2float(h), y = __high2float(h);
-                    if (e & 1) q1 = fmaf(x, x, fmaf(y, y, q1));
-                    else q0 = fmaf(x, x, fmaf(y, y, q0));
+                    q2 = fmaf(x, x, fmaf(y, y, q2));
                 }
             }
-            q0 += __shfl_xor_sync(0xffffffffu, q0, 1);
-            q0 += __shfl_xor_sync(0xffffffffu, q0, 2);
-            q1 += __shfl_xor_sync(0xffffffffu, q1, 1);
-            q1 += __shfl_xor_sync(0xffffffffu, q1, 2);
-            qn0 = sqrtf(q0);
-            qn1 = sqrtf(q1);
+            q2 += __shfl_xor_sync(0xffffffffu, q2, 1);
+            if ((tid & 1) == 0) qn_s[row] = sqrtf(q2);
+            __syncthreads();
+#pragma unroll
+            for (int j = 0; j < 8; ++j)
+#pragma unroll
+                for (int e = 0; e < 2; ++e) qn[j][e] = qn_s[8 * j + 2 * t + e];
         }
         float acc[8][4];
 #pragma unroll
         for (int j = 0; j < 8; ++j) acc[j][0] = acc[j][1] = acc[j][2] = acc[j][3] = 0.f;
 #pragma unroll
         for (int kk = 0; kk < kKs; ++kk) {
+            uint32_t ah[4], al[4];
+            const uint32_t aoff = swz64(warp * 16 + (mi & 1) * 8 + rr, 2 * kk + (mi >> 1));
+            ldmatrix_x4(hs + aoff, ah[0], ah[1], ah[2], ah[3]);
+            ldmatrix_x4(ls + aoff, al[0], al[1], al[2], al[3]);
 #pragma unroll
-            for (int jp = 0; jp < 4; ++jp) {  // n-tiles 2 jp, 2 jp + 1
-                const uint32_t off = swz64(16 * jp + (mi >> 1) * 8 + rr, 2 * kk + (mi & 1));
-                uint32_t h0, h1, h2, h3, l0, l1, l2, l3;
-                ldmatrix_x4(hs + off, h0, h1, h2, h3);
-                ldmatrix_x4(ls + off, l0, l1, l2, l3);
-                mma_m16n8k16(acc[2 * jp], a[kk], h0, h1);
-                mma_m16n8k16(acc[2 * jp], a[kk], l0, l1);
-                mma_m16n8k16(acc[2 * jp + 1], a[kk], h2, h3);
-                mma_m16n8k16(acc[2 * jp + 1], a[kk], l2, l3);
+            for (int jp = 0; jp < 4; ++jp) {  // token n-tiles 2 jp, 2 jp + 1
+                uint32_t b0, b1, b2, b3;
+                ldmatrix_x4(qs + swz64(16 * jp + (mi >> 1) * 8 + rr, 2 * kk + (mi & 1)), b0, b1, b2, b3);
+                mma_m16n8k16(acc[2 * jp], ah, b0, b1);
+                mma_m16n8k16(acc[2 * jp], al, b0, b1);
+                mma_m16n8k16(acc[2 * jp + 1], ah, b2, b3);
+                mma_m16n8k16(acc[2 * jp + 1], al, b2, b3);
             }
         }
-        // per key block: log-sum-exp of each branch over this warp's 16 rows
+        // rows g and g + 8 of the warp's tile: key blocks g0 + 16 warp + g (+ 8)
 #pragma unroll
-        for (int j = 0; j < 8; ++j) {
+        for (int h = 0; h < 2; ++h) {
+            const int col = warp * 16 + g + 8 * h;
+            const float rb = rb_s[col];
+            float vb[16], vr[16];
+            float mb = ninf, mr = ninf;
 #pragma unroll
-            for (int e = 0; e < 2; ++e) {
-                const int col = 8 * j + 2 * t + e;  // key block g0 + col
-                const int kb = g0 + col;
-                const float rb = rb_s[col];
-                const float s0 = acc[j][e], s1 = acc[j][2 + e];
-                const float b0 = v0 ? s0 * inv_sqrt_d : ninf, b1 = v1 ? s1 * inv_sqrt_d : ninf;
-                const float x0 = v0 ? fmaf(qn0, rb, s0) * inv_sqrt_d : ninf;
-                const float x1 = v1 ? fmaf(qn1, rb, s1) * inv_sqrt_d : ninf;
-                float mb = fmaxf(b0, b1), mr = fmaxf(x0, x1);
+            for (int j = 0; j < 8; ++j)
 #pragma unroll
-                for (int o = 4; o < 32; o <<= 1) {
-                    mb = fmaxf(mb, __shfl_xor_sync(0xffffffffu, mb, o));
-                    mr = fmaxf(mr, __shfl_xor_sync(0xffffffffu, mr, o));
+                for (int e = 0; e < 2; ++e) {
+                    const bool in = 8 * j + 2 * t + e < n_rows;
+                    const float sdot = acc[j][2 * h + e];
+                    vb[2 * j + e] = in ? sdot * k2 : ninf;
+                    vr[2 * j + e] = in ? fmaf(qn[j][e], rb, sdot) * k2 : ninf;
+                    mb = fmaxf(mb, vb[2 * j + e]);
+                    mr = fmaxf(mr, vr[2 * j + e]);
                 }
-                // a warp with no valid row has m = -inf: contribute (m, 0)
-                float eb = mb == ninf ? 0.f : __expf(b0 - mb) + __expf(b1 - mb);
-                float er = mr == ninf ? 0.f : __expf(x0 - mr) + __expf(x1 - mr);
+            mb = fmaxf(mb, __shfl_xor_sync(0xffffffffu, mb, 1));
+            mb = fmaxf(mb, __shfl_xor_sync(0xffffffffu, mb, 2));
+            mr = fmaxf(mr, __shfl_xor_sync(0xffffffffu, mr, 1));
+            mr = fmaxf(mr, __shfl_xor_sync(0xffffffffu, mr, 2));
+            // n_rows >= 1, so both maxima are finite here
+            float eb = 0.f, er = 0.f;
 #pragma unroll
-                for (int o = 4; o < 32; o <<= 1) {
-                    eb += __shfl_xor_sync(0xffffffffu, eb, o);
-                    er += __shfl_xor_sync(0xffffffffu, er, o);
-                }
-                if (g == 0) {
-                    float *w = red + ((warp * 64 + col) * 2) * 2;
-                    w[0] = mb;
-                    w[1] = eb;
-                    w[2] = mr;
-                    w[3] = er;
-                }
+            for (int i = 0; i < 16; ++i) {
+                eb += fast_exp2(vb[i] - mb);
+                er += fast_exp2(vr[i] - mr);
             }
-        }
-        __syncthreads();
-        if (tid < 64 && g0 + tid < p.nkb) {  // combine the four warps
-#pragma unroll
-            for (int br = 0; br < 2; ++br) {
-                float m = ninf;
-#pragma unroll
-                for (int w = 0; w < 4; ++w) m = fmaxf(m, red[((w * 64 + tid) * 2 + br) * 2]);
-                float sum = 0.f;
-#pragma unroll
-                for (int w = 0; w < 4; ++w) {
-                    const float mw = red[((w * 64 + tid) * 2 + br) * 2];
-                    if (mw != ninf) sum += red[((w * 64 + tid) * 2 + br) * 2 + 1] * __expf(mw - m);
-                }
-                (br ? sr : sb)[g0 + tid] = m + __logf(sum);
+            eb += __shfl_xor_sync(0xffffffffu, eb, 1);
+            eb += __shfl_xor_sync(0xffffffffu, eb, 2);
+            er += __shfl_xor_sync(0xffffffffu, er, 1);
+            er += __shfl_xor_sync(0xffffffffu, er, 2);
+            if (t == 0 && g0 + col < p.nkb) {
+                sb[g0 + col] = (mb + __log2f(eb)) * 0.69314718055994531f;
+                sr[g0 + col] = (mr + __log2f(er)) * 0.69314718055994531f;
             }
         }
         __syncthreads();
     }
-    __syncthreads();
     // relative masks of the row: keep where score >= row max + ln alpha
     float mb = __int_as_float(0xff800000), mr = mb;
     for (int kb = tid; kb < p.nkb; kb += blockDim.x) {
@@ -359,7 +366,7 @@ attn_status_t launch_rbs_d(const RbsArgs &a, cudaStream_t stream) {
     p.ln_alpha_base = logf(a.alpha_base);
     p.ln_alpha_rescue = logf(a.alpha_rescue);
     p.diagonal = a.diagonal;
-    const size_t smem = 3 * (size_t)64 * D * 2 + sizeof(float) * (4 * 64 * 4 + 2 * (size_t)nkb);
+    const size_t smem = 3 * (size_t)64 * D * 2 + sizeof(float) * 2 * (size_t)nkb;
     if (kernel_setup(reinterpret_cast<const void *>(rbs_scores_kernel<D>), 100 * 1024) != cudaSuccess)
         return ATTN_ERR_CUDA;
     rbs_scores_kernel<D><<<dim3(nqb, a.Hq, a.B), 128, smem, stream>>>(p);
