@@ -3,14 +3,16 @@
 // and "What mlx-arsenal ships": radius_bounded_block_scores, relative_block_mask,
 // and the recipe's union of both branches with a diagonal band).
 //
-// Three small kernels, 64-token blocks:
+// Kernels, 64-token blocks:
 //   rbs_centroid_kernel  one CTA per (key block, KV head, batch): centroid c (fp32
 //                        mean of the block's keys) and radius r = max |k - c|_2.
-//   rbs_beta_kernel      one CTA per (KV head, batch): sorts the head's radii,
-//                        takes the median and the 90th percentile (linear
-//                        interpolation between order statistics) and writes
-//                        beta = clip((r - r_low) / (r_high - r_low), 0, 1)
-//                        (1 for r > r_low, else 0, when the two coincide).
+//   rbs_beta_kernel      (only above 64 key blocks) one CTA per (KV head, batch):
+//                        sorts the head's radii, takes the median and the 90th
+//                        percentile (linear interpolation between order
+//                        statistics) and writes beta = clip((r - r_low) /
+//                        (r_high - r_low), 0, 1) (1 for r > r_low, else 0, when
+//                        the two coincide).  Up to 64 key blocks the scores kernel
+//                        does the same with one warp (warp_radius_quantiles).
 //   rbs_scores_kernel    one CTA per (query block, query head, batch): for every
 //                        key block, l_base = <q, c> / sqrt(D) and l_rescue =
 //                        (<q, c> + |q| r beta) / sqrt(D) for the block's query
@@ -19,7 +21,9 @@
 //                        either branch, or |qb - kb| < diagonal.  <q, c> for the
 //                        64 tokens and 64 key blocks at a time is a 64 x 64 x D
 //                        product on the tensor cores (warp-level bf16 MMA, fp32
-//                        accumulation) with each centroid split into a bf16 high
+//                        accumulation), taken transposed (key blocks as MMA rows)
+//                        so that each key block's log-sum-exp over the tokens stays
+//                        inside one warp, with each centroid split into a bf16 high
 //                        part and a bf16 remainder, so the two products together
 //                        carry the fp32 centroid to ~2^-17 relative (the queries
 //                        are bf16 already).
@@ -148,10 +152,49 @@ __global__ void __launch_bounds__(256)
     }
 }
 
+// Median and 90th percentile (linear interpolation between order statistics) of
+// n <= 64 radii, by one warp: bitonic sort of 64 values held two per lane (+inf
+// pads sort last), then the same arithmetic as rbs_beta_kernel.
+__device__ __forceinline__ void warp_radius_quantiles(const float *rad, int n, float &r_low,
+                                                      float &r_high) {
+    const int lane = threadIdx.x & 31;
+    const float inf = __int_as_float(0x7f800000);
+    float v0 = lane < n ? rad[lane] : inf, v1 = lane + 32 < n ? rad[lane + 32] : inf;
+    for (int k = 2; k <= 64; k <<= 1) {
+        for (int j = k >> 1; j > 0; j >>= 1) {
+            if (j == 32) {  // elements lane and lane + 32, both ascending (k = 64)
+                const float a = fminf(v0, v1), b = fmaxf(v0, v1);
+                v0 = a;
+                v1 = b;
+                continue;
+            }
+            const float p0 = __shfl_xor_sync(0xffffffffu, v0, j);
+            const float p1 = __shfl_xor_sync(0xffffffffu, v1, j);
+            const bool lower = (lane & j) == 0;
+            const bool up0 = (lane & k) == 0, up1 = ((lane + 32) & k) == 0;
+            v0 = (lower == up0) ? fminf(v0, p0) : fmaxf(v0, p0);
+            v1 = (lower == up1) ? fminf(v1, p1) : fmaxf(v1, p1);
+        }
+    }
+    auto at = [&](int i) {
+        const float a = __shfl_sync(0xffffffffu, v0, i & 31), b = __shfl_sync(0xffffffffu, v1, i & 31);
+        return i < 32 ? a : b;
+    };
+    auto quantile = [&](float q) {
+        const float pos = q * static_cast<float>(n - 1);
+        const int lo = static_cast<int>(floorf(pos));
+        const int hi = min(lo + 1, n - 1);
+        const float vlo = at(lo), vhi = at(hi);
+        return vlo + (pos - static_cast<float>(lo)) * (vhi - vlo);
+    };
+    r_low = quantile(0.5f);
+    r_high = quantile(0.9f);
+}
+
 struct ScoreParams {
     const __nv_bfloat16 *Q;
     const __nv_bfloat16 *cent_hi, *cent_lo;
-    const float *rad, *beta;
+    const float *rad, *beta;  // beta == nullptr: the kernel derives it (nkb <= 64)
     uint8_t *mask;
     float *base_out, *rescue_out;  // optional
     int Hq, Hkv, group, Sq, nqb, nkb;
@@ -195,6 +238,7 @@ __global__ void __launch_bounds__(128) rbs_scores_kernel(const ScoreParams p) {
     __shared__ float red2[2][4];
     __shared__ float rb_s[64];  // radius * beta of the key blocks of the current group
     __shared__ float qn_s[64];  // |q| of the block's tokens
+    __shared__ float quant_s[2];  // median and 90th percentile of the head's radii
     const int qb = blockIdx.x, hq = blockIdx.y, b = blockIdx.z;
     const int hkv = hq / p.group;
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -212,11 +256,41 @@ __global__ void __launch_bounds__(128) rbs_scores_kernel(const ScoreParams p) {
     // so the log-sum-exp over the tokens of a key block runs over 16 values in each
     // thread and then across the 4 lanes that share the row -- no cross-warp step.
     float qn[8][2];  // |q| of this thread's tokens 8 j + 2 t + e
+    if (!p.beta) {
+        // beta of the head's key blocks from its radii (rbs_beta_kernel's rule, here
+        // for nkb <= 64 so that the estimator needs no separate sorting launch)
+        if (warp == 0) {
+            float lo, hi;
+            warp_radius_quantiles(p.rad + hrow, p.nkb, lo, hi);
+            if (lane == 0) {
+                quant_s[0] = lo;
+                quant_s[1] = hi;
+            }
+        }
+        __syncthreads();
+    }
     for (int g0 = 0; g0 < p.nkb; g0 += 64) {
         const int nk = min(64, p.nkb - g0);
         stage64<D>(ch_tile, p.cent_hi + (hrow + g0) * D, nk);
         stage64<D>(cl_tile, p.cent_lo + (hrow + g0) * D, nk);
-        if (tid < 64) rb_s[tid] = tid < nk ? p.rad[hrow + g0 + tid] * p.beta[hrow + g0 + tid] : 0.f;
+        if (tid < 64) {
+            float rbv = 0.f;
+            if (tid < nk) {
+                const float r = p.rad[hrow + g0 + tid];
+                float bt;
+                if (p.beta) {
+                    bt = p.beta[hrow + g0 + tid];
+                } else {
+                    const float r_low = quant_s[0], r_high = quant_s[1];
+                    if (r_high > r_low)
+                        bt = fminf(fmaxf((r - r_low) / (r_high - r_low), 0.f), 1.f);
+                    else
+                        bt = r > r_low ? 1.f : 0.f;
+                }
+                rbv = r * bt;
+            }
+            rb_s[tid] = rbv;
+        }
         cp_async_wait_all();  // (the query tile's copies too, on the first group)
         __syncthreads();
         if (g0 == 0) {
@@ -343,17 +417,22 @@ attn_status_t launch_rbs_d(const RbsArgs &a, cudaStream_t stream) {
     rbs_centroid_kernel<D><<<dim3(nkb, a.Hkv, a.B), 128, 0, stream>>>(
         static_cast<const __nv_bfloat16 *>(a.K), cent_hi, cent_lo, a.rad, a.Hkv, a.Sk, nkb);
     if (cudaGetLastError() != cudaSuccess) return ATTN_ERR_CUDA;
-    int n_pow2 = 1;
-    while (n_pow2 < nkb) n_pow2 <<= 1;
-    rbs_beta_kernel<<<a.B * a.Hkv, 256, n_pow2 * sizeof(float), stream>>>(a.rad, a.beta, nkb,
-                                                                          n_pow2);
-    if (cudaGetLastError() != cudaSuccess) return ATTN_ERR_CUDA;
+    // Up to 64 key blocks the scores kernel derives beta itself (one warp sorts the
+    // head's radii); longer sequences sort in a launch of their own.
+    const bool own_beta = nkb > 64;
+    if (own_beta) {
+        int n_pow2 = 1;
+        while (n_pow2 < nkb) n_pow2 <<= 1;
+        rbs_beta_kernel<<<a.B * a.Hkv, 256, n_pow2 * sizeof(float), stream>>>(a.rad, a.beta, nkb,
+                                                                              n_pow2);
+        if (cudaGetLastError() != cudaSuccess) return ATTN_ERR_CUDA;
+    }
     ScoreParams p;
     p.Q = static_cast<const __nv_bfloat16 *>(a.Q);
     p.cent_hi = cent_hi;
     p.cent_lo = cent_lo;
     p.rad = a.rad;
-    p.beta = a.beta;
+    p.beta = own_beta ? a.beta : nullptr;
     p.mask = a.mask;
     p.base_out = a.base_scores;
     p.rescue_out = a.rescue_scores;

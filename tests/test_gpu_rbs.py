@@ -44,6 +44,8 @@ CASES = [
     (2, 2, 1, 256, 700, 64, 1.0),
     (1, 4, 4, 640, 640, 128, 0.0),
     (1, 2, 2, 1000, 1000, 128, 0.8),
+    (1, 2, 1, 200, 5000, 64, 0.8),    # 79 key blocks: two centroid groups, beta sorted apart
+    (1, 1, 1, 64, 8192, 128, 1.2),    # 128 key blocks
 ]
 
 
