@@ -122,6 +122,10 @@ attn_status_t attn_fwd_varlen(void *O, const void *Q, const void *K, const void 
  *                 1: block_mask is (B, Hq, ceil(Sq/64), ceil(Sk/64)), one matrix
  *                 per (batch, query head) -- block-sparse prefill with the
  *                 masks of attn_rbs_block_mask.
+ * A call with a block_mask and nothing else to apply (causal 0, no lengths, no
+ * document ids, no score mod, Sk <= 65536) runs the block-sparse kernel, which
+ * steps over the kept 64-key blocks of each 128-row query tile; it computes the
+ * same function.
  * Limits: Sk <= 131072.  Errors as attn_fwd, plus ATTN_ERR_INVALID for a
  * negative or non-finite softcap, softcap together with ALiBi, or only one of
  * doc_q / doc_kv, and ATTN_ERR_UNSUPPORTED for a longer Sk.
