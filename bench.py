@@ -49,6 +49,8 @@ KERNEL_SOURCES = {
                                          "gqa_attention_flash_b200/csrc/sm100_ptx.cuh"],
     "decode_split_kernel_paged": ["gqa_attention_flash_b200/csrc/attn_decode.cu",
                                   "gqa_attention_flash_b200/csrc/sm100_ptx.cuh"],
+    "attn_fwd_bsparse_kernel": ["gqa_attention_flash_b200/csrc/attn_fwd_bsparse.cu",
+                                "gqa_attention_flash_b200/csrc/sm100_ptx.cuh"],
 }
 
 
@@ -586,7 +588,8 @@ def time_block_sparse(dev, steps, warmup, peak):
             "speedup_vs_dense": t_dense / (t_est + t_sparse), "launches": steps,
             "l2": "flushed before each launch",
             "roofline": {"bound": "tensor", "achieved": tf, "peak": peak, "unit": "TFLOP/s",
-                         "frac": tf / peak, "kernel": "attn_fwd_bsparse_kernel<128>"}}
+                         "frac": tf / peak, "traffic": ncu_traffic("attn_fwd_bsparse_kernel"),
+                         "kernel": "attn_fwd_bsparse_kernel<128>"}}
 
 
 def time_backward(step, steps, warmup, peak):
