@@ -27,13 +27,20 @@
 //   buffer.  Order: S(0), dP(0), S(1), then per key tile g: [dS(g) ready]
 //   dQ += dS(g) K(g), dP(g+1), S(g+2).
 // The elementwise arithmetic runs on packed fp32 pairs (f32x2 FMA / add / mul).
-// dS is recomputed by the dQ kernel rather than reduced with atomics.  Key,
+// dS is recomputed by the dQ kernel rather than reduced with atomics.  The two
+// kernels are independent: dQ runs on a library-owned side stream forked from and
+// joined back to the caller's stream with events, so each kernel's last wave
+// overlaps the other's work (3 % on the LLM causal backward, bitwise the same).
+// The side stream and its events are shared per device; a mutex keeps the
+// fork / launch / join sequence of concurrent callers from interleaving.  Key,
 // value, query and output-gradient rows past the lengths are read as MMA
 // operands with weight exactly zero, so they must hold finite values: zero times
 // NaN or Inf is NaN, which would reach the gradients of valid rows.  The rows of
 // dQ past q_lengths and of dK, dV past k_lengths are themselves written as +0.0
 // by selection.
 #include <cuda_bf16.h>
+
+#include <mutex>
 
 #include "internal.h"
 #include "sm100_ptx.cuh"
@@ -751,6 +758,30 @@ __global__ void __launch_bounds__(kThreadsTc, 1)
     tc_teardown<C>(smem, tmem);
 }
 
+struct SideStream {
+    cudaStream_t s = nullptr;
+    cudaEvent_t fork = nullptr, join = nullptr;
+    std::mutex mu;
+};
+
+// One side stream (and its fork / join events) per device, made on first use.
+SideStream *side_stream() {
+    static std::mutex mu;
+    static SideStream *per_dev[64] = {};
+    int dev = -1;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return nullptr;
+    std::lock_guard<std::mutex> lock(mu);
+    if (!per_dev[dev]) {
+        SideStream *ss = new SideStream();
+        if (cudaStreamCreateWithFlags(&ss->s, cudaStreamNonBlocking) != cudaSuccess ||
+            cudaEventCreateWithFlags(&ss->fork, cudaEventDisableTiming) != cudaSuccess ||
+            cudaEventCreateWithFlags(&ss->join, cudaEventDisableTiming) != cudaSuccess)
+            return nullptr;
+        per_dev[dev] = ss;
+    }
+    return per_dev[dev];
+}
+
 template <int D>
 attn_status_t launch_bwd_tc_d(const BwdArgs &a, cudaStream_t stream) {
     using C = TcCfg<D>;
@@ -786,6 +817,20 @@ attn_status_t launch_bwd_tc_d(const BwdArgs &a, cudaStream_t stream) {
     p.wait_limit_ns = kWaitLimitNs;
     p.status = device_status_word();
     if (!p.status) return ATTN_ERR_CUDA;
+    const int n_qt = (a.Sq + TB - 1) / TB;
+    const long long grid = (long long)n_qt * a.Hq * a.B;
+    if (grid > 0x7fffffffll) return ATTN_ERR_INVALID;
+    // dK/dV and dQ are independent: run dQ on a side stream so that each kernel's
+    // last wave overlaps the other's work.
+    SideStream *ss = side_stream();
+    if (!ss) return ATTN_ERR_CUDA;
+    std::lock_guard<std::mutex> lock(ss->mu);
+    if (cudaEventRecord(ss->fork, stream) != cudaSuccess ||
+        cudaStreamWaitEvent(ss->s, ss->fork, 0) != cudaSuccess)
+        return ATTN_ERR_CUDA;
+    bwd_dq_tc_kernel<D><<<static_cast<unsigned>(grid), kThreadsTc, DqCfg<D>::SMEM, ss->s>>>(tq, tk, tv, tdo, p,
+                                                                                    n_qt);
+    if (cudaGetLastError() != cudaSuccess) return ATTN_ERR_CUDA;
     if (a.Sk > 0) {
         const long long grid_kv = (long long)((a.Sk + TB - 1) / TB) * a.Hkv * a.B;
         if (grid_kv > 0x7fffffffll) return ATTN_ERR_INVALID;
@@ -793,12 +838,10 @@ attn_status_t launch_bwd_tc_d(const BwdArgs &a, cudaStream_t stream) {
             tq, tk, tv, tdo, p);
         if (cudaGetLastError() != cudaSuccess) return ATTN_ERR_CUDA;
     }
-    const int n_qt = (a.Sq + TB - 1) / TB;
-    const long long grid = (long long)n_qt * a.Hq * a.B;
-    if (grid > 0x7fffffffll) return ATTN_ERR_INVALID;
-    bwd_dq_tc_kernel<D><<<static_cast<unsigned>(grid), kThreadsTc, DqCfg<D>::SMEM, stream>>>(tq, tk, tv, tdo, p,
-                                                                                     n_qt);
-    return cudaGetLastError() == cudaSuccess ? ATTN_OK : ATTN_ERR_CUDA;
+    if (cudaEventRecord(ss->join, ss->s) != cudaSuccess ||
+        cudaStreamWaitEvent(stream, ss->join, 0) != cudaSuccess)
+        return ATTN_ERR_CUDA;
+    return ATTN_OK;
 }
 
 }  // namespace

@@ -156,7 +156,10 @@ attn_status_t attn_fwd_flex(void *O, const void *Q, const void *K, const void *V
  * of dK, dV past k_lengths are +0.0).  Padding rows (Q, dO, O past q_lengths;
  * K, V past k_lengths) must hold finite values: they enter the tensor-core
  * products with weight zero, and zero times NaN or Inf is NaN.  Allocates a
- * stream-ordered workspace of B * Hq * Sq floats.  Errors as attn_fwd.
+ * stream-ordered workspace of B * Hq * Sq floats.  The dQ kernel runs on a
+ * library-owned stream forked from `stream` and joined back to it with events,
+ * so the call stays ordered on `stream` (and can be captured in a CUDA graph).
+ * Errors as attn_fwd.
  */
 attn_status_t attn_bwd(void *dQ, void *dK, void *dV, const void *dO, const void *Q, const void *K,
                        const void *V, const void *O, const float *LSE, int B, int Hq, int Hkv,
