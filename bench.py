@@ -49,6 +49,10 @@ KERNEL_SOURCES = {
                                          "gqa_attention_flash_b200/csrc/sm100_ptx.cuh"],
     "decode_split_kernel_paged": ["gqa_attention_flash_b200/csrc/attn_decode.cu",
                                   "gqa_attention_flash_b200/csrc/sm100_ptx.cuh"],
+    "attn_fwd_kernel_window": ["gqa_attention_flash_b200/csrc/attn_fwd.cu",
+                               "gqa_attention_flash_b200/csrc/sm100_ptx.cuh"],
+    "attn_fwd_kernel_image": ["gqa_attention_flash_b200/csrc/attn_fwd.cu",
+                              "gqa_attention_flash_b200/csrc/sm100_ptx.cuh"],
     "attn_fwd_bsparse_kernel": ["gqa_attention_flash_b200/csrc/attn_fwd_bsparse.cu",
                                 "gqa_attention_flash_b200/csrc/sm100_ptx.cuh"],
 }
@@ -516,7 +520,8 @@ def time_prefill_configs(dev, steps, warmup, peak, with_cpu):
         row = {"workload": w.name, "value": tf, "unit": "TFLOP/s", "ms_per_launch": ms,
                "flops_per_launch": flops, "launches": steps, "l2": "flushed before each launch",
                "roofline": {"bound": "tensor", "achieved": tf, "peak": peak, "unit": "TFLOP/s",
-                            "frac": tf / peak, "traffic": None,
+                            "frac": tf / peak,
+                            "traffic": ncu_traffic("attn_fwd_kernel_" + key) if key != "tiny" else None,
                             "kernel": f"attn_fwd_kernel<{w.D}>"}}
         if x.k_lengths is not None and key == "window":
             row["lengths"] = x.k_lengths.tolist()
@@ -765,7 +770,8 @@ def main(argv=None):
                          "the step)")
     ap.add_argument("--no-paged", action="store_true",
                     help="skip the paged-KV decode measurement (reported apart from the step)")
-    ap.add_argument("--only", choices=["prefill", "decode", "flex", "paged", "bwd"], default=None,
+    ap.add_argument("--only", choices=["prefill", "decode", "flex", "paged", "bwd", "configs"],
+                    default=None,
                     help="profiling: run one half of the step, or only the flex_attention! "
                          "workloads (no reported number)")
     ap.add_argument("--decode-batch", type=int, default=None,
@@ -793,6 +799,13 @@ def main(argv=None):
         pstep = Step(dev, "decode", args.decode_batch)
         res = time_paged(pstep, args.steps, args.warmup, peaks["hbm_gbs"])
         print(json.dumps({"profiling_run": True, "paged_ms": res["ms_per_launch"]}), flush=True)
+        return 0
+    if args.only == "configs":
+        peaks, _ = load_peaks()
+        res = time_prefill_configs(dev, args.steps, args.warmup, peaks["bf16_tflops"], False)
+        print(json.dumps({"profiling_run": True,
+                          "configs_ms": {k: v["ms_per_launch"] for k, v in res.items()}}),
+              flush=True)
         return 0
     if args.only == "bwd":
         peaks, _ = load_peaks()
