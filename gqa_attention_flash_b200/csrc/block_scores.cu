@@ -64,6 +64,8 @@ __global__ void __launch_bounds__(128)
     const int j0 = kb * kBlk, n = min(kBlk, Sk - j0);
     const __nv_bfloat16 *Kb = K + ((long long)(b * Hkv + hkv) * Sk + j0) * D;
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    // the scores kernel may start launching now (it waits for this grid's results)
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
     for (int i = tid; i < n * D / 8; i += blockDim.x)  // 16-byte copies (rows are 16B-aligned)
         cp_async16(smem_u32(kblk) + 16 * i, reinterpret_cast<const uint4 *>(Kb) + i, 16);
     cp_async_wait_all();
@@ -114,6 +116,7 @@ __global__ void __launch_bounds__(128)
 __global__ void __launch_bounds__(256)
     rbs_beta_kernel(const float *__restrict__ rad, float *__restrict__ beta, int nkb, int n_pow2) {
     extern __shared__ float v[];
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
     const long long base = (long long)blockIdx.x * nkb;
     for (int i = threadIdx.x; i < n_pow2; i += blockDim.x)
         v[i] = i < nkb ? rad[base + i] : __int_as_float(0x7f800000);  // +inf pads sort last
@@ -251,6 +254,10 @@ __global__ void __launch_bounds__(128) rbs_scores_kernel(const ScoreParams p) {
     const float ninf = __int_as_float(0xff800000);
     const uint32_t qs = smem_u32(q_tile), hs = smem_u32(ch_tile), ls = smem_u32(cl_tile);
     stage64<D>(q_tile, p.Q + ((long long)(b * p.Hq + hq) * p.Sq + i0) * D, n_rows);
+    // Launched as a programmatic dependent of the centroid (or beta) kernel: the query
+    // block above is an input of the call and is staged while that grid finishes;
+    // centroids, radii and beta are read only after it has completed.
+    asm volatile("griddepcontrol.wait;" ::: "memory");
     // The product is taken transposed, S^T = C Q^T: warp w holds the 16 key blocks
     // 16 w .. 16 w + 15 of a group (MMA rows) against all 64 tokens (MMA columns),
     // so the log-sum-exp over the tokens of a key block runs over 16 values in each
@@ -448,7 +455,20 @@ attn_status_t launch_rbs_d(const RbsArgs &a, cudaStream_t stream) {
     const size_t smem = 3 * (size_t)64 * D * 2 + sizeof(float) * 2 * (size_t)nkb;
     if (kernel_setup(reinterpret_cast<const void *>(rbs_scores_kernel<D>), 100 * 1024) != cudaSuccess)
         return ATTN_ERR_CUDA;
-    rbs_scores_kernel<D><<<dim3(nqb, a.Hq, a.B), 128, smem, stream>>>(p);
+    // programmatic dependent launch: the grid may start while the previous kernel of
+    // this call finishes (the kernel waits with griddepcontrol.wait before reading its
+    // results)
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(nqb, a.Hq, a.B);
+    cfg.blockDim = dim3(128, 1, 1);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = stream;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    if (cudaLaunchKernelEx(&cfg, rbs_scores_kernel<D>, p) != cudaSuccess) return ATTN_ERR_CUDA;
     return cudaGetLastError() == cudaSuccess ? ATTN_OK : ATTN_ERR_CUDA;
 }
 
