@@ -59,6 +59,7 @@ __global__ void __launch_bounds__(128)
                         int nkb) {
     __shared__ __align__(16) __nv_bfloat16 kblk[kBlk * D];  // the key block, read once
     __shared__ float c[D];
+    __shared__ float part[128 / (D / 2)][D];
     __shared__ float rmax_w[4];
     const int kb = blockIdx.x, hkv = blockIdx.y, b = blockIdx.z;
     const int j0 = kb * kBlk, n = min(kBlk, Sk - j0);
@@ -70,37 +71,78 @@ __global__ void __launch_bounds__(128)
         cp_async16(smem_u32(kblk) + 16 * i, reinterpret_cast<const uint4 *>(Kb) + i, 16);
     cp_async_wait_all();
     __syncthreads();
-    if (tid < D) {  // column sums on four independent chains
-        float acc[4] = {0.f, 0.f, 0.f, 0.f};
-#pragma unroll 4
-        for (int j = 0; j < n; ++j) acc[j & 3] += __bfloat162float(kblk[j * D + tid]);
-        c[tid] = ((acc[0] + acc[1]) + (acc[2] + acc[3])) / static_cast<float>(n);
+    // Keys as packed bf16 pairs; sums on packed fp32 pairs.
+    constexpr int P = D / 2;                 // column pairs per row
+    constexpr int G = 128 / P;               // row groups of the column sums
+    const uint32_t *kw = reinterpret_cast<const uint32_t *>(kblk);
+    auto bf2 = [](uint32_t u) {              // (lo, hi) bf16 -> packed fp32 pair
+        return f2_pack(__uint_as_float(u << 16), __uint_as_float(u & 0xffff0000u));
+    };
+    {
+        // column sums: thread tid sums pair tid % P over rows tid / P, + G, ...
+        const int pc = tid % P, g = tid / P;
+        uint64_t a0 = f2_pack(0.f, 0.f), a1 = f2_pack(0.f, 0.f);
+        int j = g;
+        for (; j + G < n; j += 2 * G) {
+            a0 = f2_add(a0, bf2(kw[j * P + pc]));
+            a1 = f2_add(a1, bf2(kw[(j + G) * P + pc]));
+        }
+        if (j < n) a0 = f2_add(a0, bf2(kw[j * P + pc]));
+        float lo, hi;
+        f2_unpack(f2_add(a0, a1), lo, hi);
+        part[g][2 * pc] = lo;
+        part[g][2 * pc + 1] = hi;
     }
     __syncthreads();
-    // |k - c|^2 of the warp's 16 rows (rows warp, warp + 4, ...), each lane summing
-    // its D / 32 columns; the 16 row sums are independent, so their loads and the
-    // cross-lane reductions overlap instead of running row after row
+    if (tid < D) {
+        float sum = 0.f;
+#pragma unroll
+        for (int g = 0; g < G; ++g) sum += part[g][tid];
+        c[tid] = sum / static_cast<float>(n);
+    }
+    __syncthreads();
+    // |k - c|^2 of the warp's 16 rows (rows warp, warp + 4, ...): each lane sums its
+    // column pairs (lane, lane + 32, ...) for all 16 rows, then one transposing
+    // reduction across the lanes leaves each lane with one row's total (16 shuffles
+    // instead of 5 per row)
     constexpr int kRowsPerWarp = kBlk / 4;
+    constexpr int kPairsPerLane = P / 32;
+    uint64_t cpair[kPairsPerLane];
+#pragma unroll
+    for (int q = 0; q < kPairsPerLane; ++q) cpair[q] = f2_pack(c[2 * (lane + 32 * q)], c[2 * (lane + 32 * q) + 1]);
+    const uint64_t neg1 = f2_pack(-1.f, -1.f);
     float ss[kRowsPerWarp];
 #pragma unroll
     for (int i = 0; i < kRowsPerWarp; ++i) {
         const int j = warp + 4 * i;
-        ss[i] = 0.f;
+        uint64_t acc = f2_pack(0.f, 0.f);
         if (j < n) {
 #pragma unroll
-            for (int d = lane; d < D; d += 32) {
-                const float e = __bfloat162float(kblk[j * D + d]) - c[d];
-                ss[i] = fmaf(e, e, ss[i]);
+            for (int q = 0; q < kPairsPerLane; ++q) {
+                const uint64_t e = f2_fma(cpair[q], neg1, bf2(kw[j * P + lane + 32 * q]));
+                acc = f2_fma(e, e, acc);
             }
         }
+        float lo, hi;
+        f2_unpack(acc, lo, hi);
+        ss[i] = lo + hi;  // rows past n hold 0
     }
+    // transposing reduction: after the step with lane bit m, a lane keeps the rows
+    // whose index bit matches its lane bit and adds its partner's partial sums
 #pragma unroll
-    for (int o = 16; o > 0; o >>= 1)
+    for (int half = kRowsPerWarp / 2, bitl = 16; half >= 1; half >>= 1, bitl >>= 1) {
+        const bool up = (lane & bitl) != 0;
 #pragma unroll
-        for (int i = 0; i < kRowsPerWarp; ++i) ss[i] += __shfl_xor_sync(0xffffffffu, ss[i], o);
-    float rm = 0.f;
+        for (int i = 0; i < half; ++i) {
+            const float send = up ? ss[i] : ss[i + half];
+            const float keep = up ? ss[i + half] : ss[i];
+            ss[i] = keep + __shfl_xor_sync(0xffffffffu, send, bitl);
+        }
+    }
+    float tot = ss[0] + __shfl_xor_sync(0xffffffffu, ss[0], 1);  // lanes 2r, 2r + 1 hold one row
+    float rm = sqrtf(tot);
 #pragma unroll
-    for (int i = 0; i < kRowsPerWarp; ++i) rm = fmaxf(rm, sqrtf(ss[i]));  // rows past n hold 0
+    for (int o = 2; o < 32; o <<= 1) rm = fmaxf(rm, __shfl_xor_sync(0xffffffffu, rm, o));
     if (lane == 0) rmax_w[warp] = rm;
     const long long row = (long long)(b * Hkv + hkv) * nkb + kb;
     if (tid < D) {  // the centroid as bf16 high part + bf16 remainder
