@@ -1,6 +1,7 @@
 // attn_api.cu -- the library's C ABI (declared in include/gqa_attn.h):
 // host-side argument validation, TMA descriptor encoding, the per-device status
 // word, and the workspaces (from a per-device pool the library owns).
+#include <nvtx3/nvToolsExt.h>
 #include <cmath>
 #include <cstdint>
 #include <cstring>
@@ -183,6 +184,17 @@ attn_status_t launch_wait_probe(int limit_us, cudaStream_t stream) {
 using namespace gqa;
 
 namespace {
+// NVTX range around an ABI call (host side: the enqueue of its kernels), so that
+// a profiler's timeline names the calls; no cost without a tool attached.
+struct NvtxRange {
+    explicit NvtxRange(const char *name) { nvtxRangePushA(name); }
+    ~NvtxRange() { nvtxRangePop(); }
+    NvtxRange(const NvtxRange &) = delete;
+    NvtxRange &operator=(const NvtxRange &) = delete;
+};
+}  // namespace
+
+namespace {
 
 attn_status_t validate_fwd(void *O, const void *Q, const void *K, const void *V, float *LSE, int B,
                            int Hq, int Hkv, int Sq, int Sk, int D, float scale, int causal,
@@ -215,6 +227,7 @@ attn_status_t attn_fwd_varlen(void *O, const void *Q, const void *K, const void 
                               int B, int Hq, int Hkv, int Sq, int Sk, int D, float scale,
                               int causal, int window, int input_pos, const int32_t *k_lengths,
                               const int32_t *q_lengths, void *stream) {
+    NvtxRange nvtx_range("attn_fwd_varlen");
     attn_status_t st =
         validate_fwd(O, Q, K, V, LSE, B, Hq, Hkv, Sq, Sk, D, scale, causal, window, input_pos);
     if (st != ATTN_OK) return st;
@@ -250,6 +263,7 @@ attn_status_t attn_fwd_varlen(void *O, const void *Q, const void *K, const void 
 attn_status_t attn_fwd(void *O, const void *Q, const void *K, const void *V, float *LSE, int B,
                        int Hq, int Hkv, int Sq, int Sk, int D, float scale, int causal, int window,
                        int input_pos, const int32_t *k_lengths, void *stream) {
+    NvtxRange nvtx_range("attn_fwd");
     return attn_fwd_varlen(O, Q, K, V, LSE, B, Hq, Hkv, Sq, Sk, D, scale, causal, window,
                            input_pos, k_lengths, nullptr, stream);
 }
@@ -261,6 +275,7 @@ attn_status_t attn_fwd_flex(void *O, const void *Q, const void *K, const void *V
                             float softcap, const float *alibi_slopes,
                             const int32_t *doc_q, const int32_t *doc_kv,
                             const uint8_t *block_mask, int block_mask_per_head, void *stream) {
+    NvtxRange nvtx_range("attn_fwd_flex");
     attn_status_t st =
         validate_fwd(O, Q, K, V, LSE, B, Hq, Hkv, Sq, Sk, D, scale, causal, window, input_pos);
     if (st != ATTN_OK) return st;
@@ -312,6 +327,7 @@ attn_status_t attn_fwd_flex(void *O, const void *Q, const void *K, const void *V
 attn_status_t attn_decode(void *O, const void *Q, const void *K, const void *V,
                           const int32_t *lengths, int n_splits, void *stream, int B, int Hq,
                           int Hkv, int S_cap, int D) {
+    NvtxRange nvtx_range("attn_decode");
     if (B < 0 || Hq < 1 || Hkv < 1 || S_cap < 0 || n_splits < 1 || n_splits > 64)
         return ATTN_ERR_INVALID;
     if (Hq % Hkv != 0 || Hq / Hkv > 16) return ATTN_ERR_INVALID;
@@ -349,6 +365,7 @@ attn_status_t attn_bwd(void *dQ, void *dK, void *dV, const void *dO, const void 
                        const void *V, const void *O, const float *LSE, int B, int Hq, int Hkv,
                        int Sq, int Sk, int D, float scale, int causal, int window, int input_pos,
                        const int32_t *k_lengths, const int32_t *q_lengths, void *stream) {
+    NvtxRange nvtx_range("attn_bwd");
     attn_status_t st =
         validate_fwd(const_cast<void *>(O), Q, K, V, nullptr, B, Hq, Hkv, Sq, Sk, D, scale, causal,
                      window, input_pos);
@@ -403,6 +420,7 @@ attn_status_t attn_rbs_block_mask(uint8_t *block_mask, float *base_scores, float
                                   const void *Q, const void *K, int B, int Hq, int Hkv, int Sq,
                                   int Sk, int D, float alpha_base, float alpha_rescue,
                                   int diagonal, void *stream) {
+    NvtxRange nvtx_range("attn_rbs_block_mask");
     if (B < 0 || Hq < 1 || Hkv < 1 || Sq < 0 || Sk < 0 || diagonal < 0) return ATTN_ERR_INVALID;
     if (Hq % Hkv != 0) return ATTN_ERR_INVALID;
     if (!(alpha_base > 0.f) || !(alpha_rescue > 0.f) || !std::isfinite(alpha_base) ||
@@ -447,6 +465,7 @@ attn_status_t attn_decode_paged(void *O, const void *Q, const void *K_cache, con
                                 const int32_t *block_tables, const int32_t *seq_lens, int n_splits,
                                 void *stream, int B, int Hq, int Hkv, int num_blocks,
                                 int block_size, int max_blocks_per_seq, int D) {
+    NvtxRange nvtx_range("attn_decode_paged");
     if (B < 0 || Hq < 1 || Hkv < 1 || num_blocks < 1 || max_blocks_per_seq < 0 || n_splits < 1 ||
         n_splits > 64)
         return ATTN_ERR_INVALID;

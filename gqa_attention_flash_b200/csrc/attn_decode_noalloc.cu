@@ -23,6 +23,7 @@
 // address is looked up with cudaGetSymbolAddress, once per device, on the first
 // call made while that device is current; that first call should come before
 // any stream capture begins.
+#include <nvtx3/nvToolsExt.h>
 #include <mutex>
 
 #include <cuda_runtime.h>
@@ -67,6 +68,11 @@ using namespace gqa;
 extern "C" attn_status_t attn_decode_noalloc(void *O, const void *Q, const void *K, const void *V,
                                              const int32_t *lengths, int n_splits, void *stream,
                                              int B, int Hq, int Hkv, int S_cap, int D) {
+    // NVTX range around the call (host side), as for the other entry points
+    nvtxRangePushA("attn_decode_noalloc");
+    struct Pop {
+        ~Pop() { nvtxRangePop(); }
+    } pop_at_return;
     // Same argument checks as attn_decode.
     if (B < 0 || Hq < 1 || Hkv < 1 || S_cap < 0 || n_splits < 1 || n_splits > 64)
         return ATTN_ERR_INVALID;

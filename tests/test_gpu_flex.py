@@ -175,7 +175,7 @@ def test_full_size_flex_workloads(orc, key):
     if doc is not None:
         starts = np.flatnonzero(np.diff(doc.numpy())) + 1
         extra = tuple(starts) + tuple(starts - 1)
-    rows = sample_rows(w.S, seed=w.seed, n_random=12, extra=extra)
+    rows = sample_rows(w.S, seed=w.seed, n_random=512, extra=extra)
     Or, Lr = orc.flex_fwd(Q[:, :, torch.as_tensor(rows, dtype=torch.long)].double().numpy(),
                           K.double().numpy(), V.double().numpy(), w.scale, causal=w.causal,
                           rows=rows, Sq=w.S, softcap=w.softcap,

@@ -87,7 +87,8 @@ def test_nan_beyond_k_lengths_ignored(orc):
 @pytest.mark.parametrize("name", ["llm", "window", "image"])
 def test_full_size_sampled(orc, name):
     """Full-size workloads in the benchmark's launch configuration, compared on
-    sampled query rows (all batches and heads) including tile and mask edges."""
+    sampled query rows (all batches and heads): 512 random rows plus tile and mask
+    edges."""
     w = W.PREFILL_WORKLOADS[name]
     x = W.make_prefill(w)
     O, L = gpu_prefill(x.Q, x.K, x.V, w.scale, w.causal, w.window, w.input_pos, x.k_lengths,
@@ -96,7 +97,7 @@ def test_full_size_sampled(orc, name):
     if x.k_lengths is not None:
         for v in x.k_lengths.tolist():
             extra += [v - 1, v, v - w.window, v - w.window + 1]
-    rows = sample_rows(w.Sq, 5, n_random=12, extra=extra)
+    rows = sample_rows(w.Sq, 5, n_random=512, extra=extra)
     Or, Lr = oracle_prefill(orc, x.Q, x.K, x.V, w.scale, w.causal, w.window, w.input_pos,
                             x.k_lengths, x.q_lengths, rows=rows)
     compare(O, L, Or, Lr, rows=rows, what=name)
