@@ -139,3 +139,20 @@ def test_one_hot_probe_bit_exact(orc, case):
             assert np.array_equal(got[:, h], want[:, h]), \
                 f"{case} run {run} head {h} (chunk {run * Hkv + h // G})"
         compare(O.cpu(), L.cpu(), Or, Lr, what=f"{case} run {run}")
+
+
+@pytest.mark.parametrize("Sk", [65499, 65617])
+def test_longest_key_sequences(orc, Sk):
+    """1024 key blocks (the last one ragged), the most the block-sparse kernel's per-CTA
+    list holds, and two blocks more (the call then runs on the flex kernel's list
+    path): the same function."""
+    B, Hq, Hkv, Sq, D = 1, 2, 1, 200, 128
+    Q, K, V = W.random_prefill(99, B, Hq, Hkv, Sq, Sk, D)
+    mask = random_block_mask(98, B, Hq, Sq, Sk, 0.05, True)
+    # the last key block is kept by one query block, so the ragged end of the keys is visited
+    mask[0, 0, 0, -1] = 2
+    scale = 1.0 / math.sqrt(D)
+    O, L = gpu_block_sparse(Q, K, V, scale, mask)
+    Or, Lr = orc.flex_fwd(Q.double().numpy(), K.double().numpy(), V.double().numpy(), scale,
+                          block_keep=keep_flags(mask, B, Hq))
+    compare(O, L, Or, Lr, what=f"Sk {Sk}")
