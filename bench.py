@@ -49,6 +49,11 @@ KERNEL_SOURCES = {
                                          "gqa_attention_flash_b200/csrc/sm100_ptx.cuh"],
     "decode_split_kernel_paged": ["gqa_attention_flash_b200/csrc/attn_decode.cu",
                                   "gqa_attention_flash_b200/csrc/sm100_ptx.cuh"],
+    "attn_fwd_kernel_flex_alibi": ["gqa_attention_flash_b200/csrc/attn_fwd.cu",
+                                   "gqa_attention_flash_b200/csrc/sm100_ptx.cuh"],
+    "attn_bwd": ["gqa_attention_flash_b200/csrc/attn_bwd.cu",
+                 "gqa_attention_flash_b200/csrc/attn_bwd_tc.cu",
+                 "gqa_attention_flash_b200/csrc/sm100_ptx.cuh"],
     "attn_fwd_kernel_window": ["gqa_attention_flash_b200/csrc/attn_fwd.cu",
                                "gqa_attention_flash_b200/csrc/sm100_ptx.cuh"],
     "attn_fwd_kernel_image": ["gqa_attention_flash_b200/csrc/attn_fwd.cu",
@@ -631,7 +636,7 @@ def time_backward(step, steps, warmup, peak):
     return {"workload": w.name + ", backward", "value": tf, "unit": "TFLOP/s",
             "ms_per_launch": ms, "flops_per_launch": flops, "launches": steps,
             "roofline": {"bound": "tensor", "achieved": tf, "peak": peak, "unit": "TFLOP/s",
-                         "frac": tf / peak,
+                         "frac": tf / peak, "traffic": ncu_traffic("attn_bwd"),
                          "kernel": "bwd_dkdv_tc_kernel<128> + bwd_dq_tc_kernel<128> + bwd_delta_kernel<128>"}}
 
 
