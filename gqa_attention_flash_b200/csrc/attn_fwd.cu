@@ -722,10 +722,17 @@ __global__ void __launch_bounds__(kThreads, 1)
                             if (st == 1 && p.doc_kv) {  // uniform: st depends on the warp only
                                 const int kc = kv0 + 32 * j + lane;
                                 const int dv = kc < p.Sk ? p.doc_kv[kc] : 0;
+                                const int dv0 = __shfl_sync(0xffffffffu, dv, 0);
                                 uint32_t same = 0;
+                                if (__all_sync(0xffffffffu, dv == dv0)) {
+                                    // the 32 keys belong to one document (packed documents
+                                    // leave most chunks so): one compare for the row
+                                    same = dv0 == doc_row ? 0xffffffffu : 0u;
+                                } else {
 #pragma unroll 1
-                                for (int c = 0; c < 32; ++c)
-                                    same |= (__shfl_sync(0xffffffffu, dv, c) == doc_row ? 1u : 0u) << c;
+                                    for (int c = 0; c < 32; ++c)
+                                        same |= (__shfl_sync(0xffffffffu, dv, c) == doc_row ? 1u : 0u) << c;
+                                }
                                 m &= same;
                             }
                             vm[j] = m;
