@@ -140,6 +140,22 @@ __global__ void __launch_bounds__(kDecThreads)
         if (lane == 0) {
             prefetch_tensormap(&tmK);
             prefetch_tensormap(&tmV);
+            // paged: block ids of a tile's chunks, loaded one tile ahead so that the
+            // block-table reads overlap the previous tile's copies instead of each
+            // copy waiting for its own read (block_size >= 8: at most TN / 8 chunks)
+            constexpr int kMaxChunks = TN / 8;
+            int ids[kMaxChunks];
+            auto load_ids = [&](int it2) {
+                if constexpr (kPaged) {
+                    const int row2 = (t_begin + it2) * TN;
+                    const int n2 = (min(TN, len - row2) + p.box_rows - 1) / p.box_rows;
+                    const int32_t *bt = p.block_tables + (long long)b * p.max_blocks;
+#pragma unroll
+                    for (int k = 0; k < kMaxChunks; ++k)
+                        ids[k] = k < n2 ? bt[(row2 + k * p.box_rows) >> p.block_shift] : 0;
+                }
+            };
+            if (n_tiles > 0) load_ids(0);
             for (int it = 0; it < n_tiles; ++it) {
                 const int st = it % C::NS;
                 const int use = it / C::NS;
@@ -167,11 +183,16 @@ __global__ void __launch_bounds__(kDecThreads)
                     // consumers mask those keys and zero those V rows.
                     const int br = p.box_rows;
                     const int n_chunks = (min(TN, len - row) + br - 1) / br;
+                    int cur[kMaxChunks];
+#pragma unroll
+                    for (int k = 0; k < kMaxChunks; ++k) cur[k] = ids[k];
+                    if (it + 1 < n_tiles) load_ids(it + 1);
                     mbar_arrive_expect_tx(full(st), 2 * n_chunks * br * 128 * C::NBOX);
-                    const int32_t *bt = p.block_tables + (long long)b * p.max_blocks;
-                    for (int k = 0; k < n_chunks; ++k) {
+#pragma unroll
+                    for (int k = 0; k < kMaxChunks; ++k) {
+                        if (k >= n_chunks) break;
                         const int j = row + k * br;
-                        const int blk = bt[j >> p.block_shift];
+                        const int blk = cur[k];
                         if (blk < 0 || blk >= p.num_blocks) record_status(p.status, ATTN_ERR_DEVICE_BOUNDS);
                         // an out-of-range block reads as zeros (outside the tensor map)
                         const int prow = blk * (1 << p.block_shift) + (j & ((1 << p.block_shift) - 1));
