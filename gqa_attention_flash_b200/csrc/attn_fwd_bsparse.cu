@@ -323,58 +323,68 @@ __global__ void __launch_bounds__(kSpThreads, 2)
                 ok = false;
                 break;
             }
-            tc_fence_after();
-            uint32_t sr[2][32];
-            tmem_ld32(s_addr, sr[0]);
-            tmem_ld32(s_addr + 32, sr[1]);
-            tmem_wait_ld();
-            reg_fence32(sr[0]);
-            reg_fence32(sr[1]);
-            float *s = reinterpret_cast<float *>(&sr[0][0]);
-            if (c_hi < SP_BN) {
-#pragma unroll
-                for (int c = 0; c < SP_BN; ++c) s[c] = c < c_hi ? s[c] : sp_neg_inf();
-            }
-            // online softmax in the exp2 domain; O is rescaled only when the row max
-            // grows by more than 2^8
-            // row max: four independent chains of three-input maxima
-            float mx[4];
-#pragma unroll
-            for (int g = 0; g < 4; ++g) {
-                float a = fmax3(s[16 * g], s[16 * g + 1], s[16 * g + 2]);
-#pragma unroll
-                for (int c = 16 * g + 3; c < 16 * g + 15; c += 2) a = fmax3(a, s[c], s[c + 1]);
-                mx[g] = fmaxf(a, s[16 * g + 15]);
-            }
-            const float m_new = fmax3(mx[0], mx[1], fmaxf(mx[2], mx[3])) * sl2;
             float alpha = 1.f;
             bool resc = false;
-            if (m_new > m_used + 8.f) {
-                alpha = fast_exp2(m_used - m_new);
-                m_used = m_new;
-                resc = true;
-            }
-            const float neg_m = (m_used == sp_neg_inf()) ? 0.f : -m_used;
-            const uint64_t sl2x2 = f2_pack(sl2, sl2), negm2 = f2_pack(neg_m, neg_m);
-            uint64_t sum2 = f2_pack(0.f, 0.f);
+            if (c_hi == 0) {
+                // this row's query block does not keep the key block (the other one
+                // does): every score is masked, so P = 0 and m, l stay as they are --
+                // the same bits the full pass below would produce, without its work
+                const uint32_t z[16] = {0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u};
+                tc_fence_after();  // after S_j has landed in these columns
+                tmem_st16(s_addr, z);
+                tmem_st16(s_addr + 16, z);
+            } else {
+                tc_fence_after();
+                uint32_t sr[2][32];
+                tmem_ld32(s_addr, sr[0]);
+                tmem_ld32(s_addr + 32, sr[1]);
+                tmem_wait_ld();
+                reg_fence32(sr[0]);
+                reg_fence32(sr[1]);
+                float *s = reinterpret_cast<float *>(&sr[0][0]);
+                if (c_hi < SP_BN) {
 #pragma unroll
-            for (int c = 0; c < 2; ++c) {
-                uint32_t pk[16];
-#pragma unroll
-                for (int k = 0; k < 16; ++k) {
-                    float x0, x1;
-                    f2_unpack(f2_fma(f2_pack(s[c * 32 + 2 * k], s[c * 32 + 2 * k + 1]), sl2x2, negm2),
-                              x0, x1);
-                    const float p0 = fast_exp2(x0);
-                    const float p1 = fast_exp2(x1);
-                    sum2 = f2_add(sum2, f2_pack(p0, p1));
-                    pk[k] = pack_bf16x2(p0, p1);
+                    for (int c = 0; c < SP_BN; ++c) s[c] = c < c_hi ? s[c] : sp_neg_inf();
                 }
-                tmem_st16(s_addr + c * 16, pk);
+                // online softmax in the exp2 domain; O is rescaled only when the row max
+                // grows by more than 2^8
+                // row max: four independent chains of three-input maxima
+                float mx[4];
+#pragma unroll
+                for (int g = 0; g < 4; ++g) {
+                    float a = fmax3(s[16 * g], s[16 * g + 1], s[16 * g + 2]);
+#pragma unroll
+                    for (int c = 16 * g + 3; c < 16 * g + 15; c += 2) a = fmax3(a, s[c], s[c + 1]);
+                    mx[g] = fmaxf(a, s[16 * g + 15]);
+                }
+                const float m_new = fmax3(mx[0], mx[1], fmaxf(mx[2], mx[3])) * sl2;
+                if (m_new > m_used + 8.f) {
+                    alpha = fast_exp2(m_used - m_new);
+                    m_used = m_new;
+                    resc = true;
+                }
+                const float neg_m = (m_used == sp_neg_inf()) ? 0.f : -m_used;
+                const uint64_t sl2x2 = f2_pack(sl2, sl2), negm2 = f2_pack(neg_m, neg_m);
+                uint64_t sum2 = f2_pack(0.f, 0.f);
+#pragma unroll
+                for (int c = 0; c < 2; ++c) {
+                    uint32_t pk[16];
+#pragma unroll
+                    for (int k = 0; k < 16; ++k) {
+                        float x0, x1;
+                        f2_unpack(f2_fma(f2_pack(s[c * 32 + 2 * k], s[c * 32 + 2 * k + 1]), sl2x2, negm2),
+                                  x0, x1);
+                        const float p0 = fast_exp2(x0);
+                        const float p1 = fast_exp2(x1);
+                        sum2 = f2_add(sum2, f2_pack(p0, p1));
+                        pk[k] = pack_bf16x2(p0, p1);
+                    }
+                    tmem_st16(s_addr + c * 16, pk);
+                }
+                float sum0, sum1;
+                f2_unpack(sum2, sum0, sum1);
+                l = l * alpha + (sum0 + sum1);
             }
-            float sum0, sum1;
-            f2_unpack(sum2, sum0, sum1);
-            l = l * alpha + (sum0 + sum1);
             // P_{j-1} V_{j-1} must be complete before O is rescaled, and before P_j is
             // handed over (this also keeps every barrier below one phase ahead at most).
             if (j > 0) {
