@@ -60,9 +60,14 @@ def rbs_inputs(case, seed):
     return Q, K, V
 
 
-@pytest.mark.parametrize("case", CASES, ids=[str(c) for c in CASES])
+# Scores only: up to 64 key blocks, more query blocks than one wave of scores CTAs
+# holds one each, so a CTA scores several in turn (with the next one's load in flight).
+SCORE_CASES = CASES + [(1, 8, 2, 8192, 4096, 64, 0.8), (2, 16, 4, 4096, 4096, 128, 1.0)]
+
+
+@pytest.mark.parametrize("case", SCORE_CASES, ids=[str(c) for c in SCORE_CASES])
 def test_rbs_scores_and_mask(orc, case):
-    Q, K, V = rbs_inputs(case, 50 + CASES.index(case))
+    Q, K, V = rbs_inputs(case, 50 + SCORE_CASES.index(case))
     mask, base, resc = gpu_rbs(Q, K)
     ob, orr = orc.rbs_block_scores(Q.double().numpy(), K.double().numpy())
     assert np.max(np.abs(base - ob)) <= SCORE_TOL, np.max(np.abs(base - ob))
