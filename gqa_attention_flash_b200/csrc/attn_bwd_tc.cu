@@ -20,7 +20,11 @@
 //   TMEM (512 columns): S^T | dP^T | dV | dK.
 //   Tensor-pipe order per ring item t: dP^T(t), [P^T(t) ready] dV += P^T dO,
 //   S^T(t+1), [dS^T(t) ready] dK += dS^T Q -- so P^T(t+1) is computed while dK(t)
-//   and dP^T(t+1) run, and dS^T(t) while dV(t) and S^T(t+1) run.
+//   and dP^T(t+1) run, and dS^T(t) while dV(t) and S^T(t+1) run.  P^T is released
+//   in two halves: each elementwise warp stores and signals the first 32 of its 64
+//   query columns before it computes the other 32, and dV issues the K-steps of
+//   the first halves (query columns 0-31, 64-95) while the rest is computed (4 %
+//   faster on the LLM causal backward than one release).
 // bwd_dq_tc_kernel: one CTA per (128-row query tile, query head, batch), same
 //   roles over the visible 128-key tiles, Q and dO resident, K in a 3-slot and V
 //   in a 2-slot ring; TMEM: S0 | S1 | dP | dQ, dS (bf16) written over its own S
@@ -72,12 +76,12 @@ struct TcCfg {
     __host__ __device__ static constexpr int stage(int s) { return OFF_S + s * STAGE; }
     static constexpr int OFF_BAR = OFF_S + NS * STAGE;
     // barriers: resident; per ring slot full / empty of its Q half and of its dO
-    // half (they are released at different points); s_full, dp_full, p_done,
-    // ds_full, done
+    // half (they are released at different points); s_full, dp_full, p_done (first
+    // half of P^T), ds_full, done, p_done2 (second half of P^T)
     static constexpr int BAR_RES = 0, BAR_FULLQ = 1, BAR_EMPTYQ = 1 + NS, BAR_FULLD = 1 + 2 * NS,
                          BAR_EMPTYD = 1 + 3 * NS, BAR_SFULL = 1 + 4 * NS, BAR_DPFULL = 2 + 4 * NS,
                          BAR_PDONE = 3 + 4 * NS, BAR_DSFULL = 4 + 4 * NS, BAR_DONE = 5 + 4 * NS,
-                         N_BARS = 6 + 4 * NS;
+                         BAR_PDONE2 = 6 + 4 * NS, N_BARS = 7 + 4 * NS;
     static constexpr int OFF_MISC = OFF_BAR + N_BARS * 8;
     static constexpr int SMEM = OFF_MISC + 16 + 1024;
     // TMEM columns
@@ -181,6 +185,24 @@ __device__ __forceinline__ void mma_tmem_a(uint32_t d_tmem, uint32_t a_tmem, uin
     }
 }
 
+// Half r of the K-steps of mma_tmem_a<D, true>: K-steps 4 k + 2 r, 4 k + 2 r + 1 (k = 0, 1),
+// i.e. A's K index 32 r .. 32 r + 31 and 64 + 32 r .. 64 + 32 r + 31.
+template <int D>
+__device__ __forceinline__ void mma_tmem_a_half(uint32_t d_tmem, uint32_t a_tmem, uint32_t b_smem,
+                                                bool accumulate, int r) {
+    using C = TcCfg<D>;
+    constexpr uint32_t id = idesc_bf16_f32(TB, D, 0, 1);
+#pragma unroll
+    for (int k = 0; k < 2; ++k)
+#pragma unroll
+        for (int e = 0; e < 2; ++e) {
+            const int kk = 4 * k + 2 * r + e;
+            const uint32_t a_col = (kk >> 2) * 64 + (kk & 3) * 8;
+            mma_ts(d_tmem, a_tmem + a_col, smem_desc_sw128(b_smem + kk * 16 * 128, C::BOX, 1024), id,
+                   (accumulate || kk > 0) ? 1u : 0u);
+        }
+}
+
 // Shared set-up: barriers (the elementwise warps' arrival barriers count 256
 // arrivals, the others one), TMEM allocation (warp 9), 512 columns.
 template <class C>
@@ -190,7 +212,7 @@ __device__ __forceinline__ uint32_t tc_setup(uint8_t *smem, uint32_t sbase) {
     if (threadIdx.x == 0) {
         for (int i = 0; i < C::N_BARS; ++i)
             mbar_init(sbase + C::OFF_BAR + 8 * i,
-                      (i == C::BAR_PDONE || i == C::BAR_DSFULL) ? kEltThreads : 1);
+                      (i == C::BAR_PDONE || i == C::BAR_PDONE2 || i == C::BAR_DSFULL) ? kEltThreads : 1);
         *abort_flag = 0;
         fence_mbar_init();
     }
@@ -379,10 +401,16 @@ __global__ void __launch_bounds__(kThreadsTc, 1)
                 tc_fence_after();
                 mma_kmajor<D>(tmem + C::COL_DP, sbase + C::OFF_R1, do_s);  // dP^T = V dO^T
                 mma_commit(bar(C::BAR_DPFULL));
+                // dV += P^T dO in two halves of its K-steps: the query columns 0-31 and
+                // 64-95 of P^T are released first, 32-63 and 96-127 after them
                 if (!(ok = mbar_wait(bar(C::BAR_PDONE), it & 1, abort_flag, p.wait_limit_ns, p.status)))
                     break;
                 tc_fence_after();
-                mma_tmem_a<D, true>(tmem + C::COL_A, tmem + C::COL_S, do_s, it > 0);  // dV += P^T dO
+                mma_tmem_a_half<D>(tmem + C::COL_A, tmem + C::COL_S, do_s, it > 0, 0);
+                if (!(ok = mbar_wait(bar(C::BAR_PDONE2), it & 1, abort_flag, p.wait_limit_ns, p.status)))
+                    break;
+                tc_fence_after();
+                mma_tmem_a_half<D>(tmem + C::COL_A, tmem + C::COL_S, do_s, true, 1);
                 mma_commit(bar(C::BAR_EMPTYD + st));
                 if (it + 1 < n_it) {
                     const int st1 = (it + 1) % C::NS;
@@ -437,33 +465,35 @@ __global__ void __launch_bounds__(kThreadsTc, 1)
                 // exponent arguments on packed fp32 pairs (rows[] holds -LSE * log2 e)
                 const float4 *l4 = reinterpret_cast<const float4 *>(rows + cb);
                 const uint64_t sl2x2 = f2_pack(p.scale_log2, p.scale_log2);
+                // two halves of the warp's 64 columns, each released to the dV product as
+                // soon as it is in TMEM
 #pragma unroll
-                for (int q = 0; q < 16; ++q) {
-                    const float4 l = l4[q];
+                for (int c = 0; c < 2; ++c) {
 #pragma unroll
-                    for (int h = 0; h < 2; ++h) {
-                        const int x = 4 * q + 2 * h;
-                        float x0, x1;
-                        f2_unpack(f2_fma(f2_pack(__uint_as_float(sv[x >> 5][x & 31]),
-                                                 __uint_as_float(sv[x >> 5][(x + 1) & 31])),
-                                         sl2x2, h ? f2_pack(l.z, l.w) : f2_pack(l.x, l.y)),
-                                  x0, x1);
-                        const float v0 = fast_exp2(x0), v1 = fast_exp2(x1);
-                        pr[x] = (x >= lo && x < hi) ? v0 : 0.f;
-                        pr[x + 1] = (x + 1 >= lo && x + 1 < hi) ? v1 : 0.f;
+                    for (int q = 8 * c; q < 8 * c + 8; ++q) {
+                        const float4 l = l4[q];
+#pragma unroll
+                        for (int h = 0; h < 2; ++h) {
+                            const int x = 4 * q + 2 * h;
+                            float x0, x1;
+                            f2_unpack(f2_fma(f2_pack(__uint_as_float(sv[x >> 5][x & 31]),
+                                                     __uint_as_float(sv[x >> 5][(x + 1) & 31])),
+                                             sl2x2, h ? f2_pack(l.z, l.w) : f2_pack(l.x, l.y)),
+                                      x0, x1);
+                            const float v0 = fast_exp2(x0), v1 = fast_exp2(x1);
+                            pr[x] = (x >= lo && x < hi) ? v0 : 0.f;
+                            pr[x + 1] = (x + 1 >= lo && x + 1 < hi) ? v1 : 0.f;
+                        }
                     }
+                    uint32_t pk[16];
+#pragma unroll
+                    for (int k = 0; k < 16; ++k) pk[k] = pack_bf16x2(pr[32 * c + 2 * k], pr[32 * c + 2 * k + 1]);
+                    tmem_st16(trow + C::COL_S + cb + 16 * c, pk);
+                    tmem_wait_st();
+                    tc_fence_before();
+                    mbar_arrive(bar(c ? C::BAR_PDONE2 : C::BAR_PDONE));
                 }
             }
-#pragma unroll
-            for (int c = 0; c < 2; ++c) {
-                uint32_t pk[16];
-#pragma unroll
-                for (int k = 0; k < 16; ++k) pk[k] = pack_bf16x2(pr[32 * c + 2 * k], pr[32 * c + 2 * k + 1]);
-                tmem_st16(trow + C::COL_S + cb + 16 * c, pk);
-            }
-            tmem_wait_st();
-            tc_fence_before();
-            mbar_arrive(bar(C::BAR_PDONE));
             if (!warp_wait(bar(C::BAR_DPFULL), it & 1, abort_flag, p.wait_limit_ns, p.status)) {
                 ok = false;
                 break;
@@ -538,7 +568,8 @@ struct DqCfg {
     static constexpr int BAR_RES = 0, BAR_FULLK = 1, BAR_EMPTYK = 1 + NK, BAR_FULLV = 1 + 2 * NK,
                          BAR_EMPTYV = 1 + 2 * NK + NV, BAR_SFULL = 1 + 2 * NK + 2 * NV,  // two
                          BAR_DPFULL = 3 + 2 * NK + 2 * NV, BAR_DSFULL = 4 + 2 * NK + 2 * NV,
-                         BAR_DONE = 5 + 2 * NK + 2 * NV, BAR_PDONE = -1, N_BARS = 6 + 2 * NK + 2 * NV;
+                         BAR_DONE = 5 + 2 * NK + 2 * NV, BAR_PDONE = -1, BAR_PDONE2 = -1,
+                         N_BARS = 6 + 2 * NK + 2 * NV;
     static constexpr int OFF_MISC = OFF_BAR + N_BARS * 8;
     static constexpr int SMEM = OFF_MISC + 16 + 1024;
     // TMEM: two S buffers (dS written over its own S), dP, dQ
