@@ -155,6 +155,20 @@ attn_status_t make_tmap_bf16_paged(CUtensorMap *map, const void *base, uint64_t 
     return r == CUDA_SUCCESS ? ATTN_OK : ATTN_ERR_INVALID;
 }
 
+attn_status_t make_tmap_bf16_paged_wide(CUtensorMap *map, const void *base, uint64_t heads,
+                                        uint64_t rows, uint32_t box_rows) {
+    EncodeTiledFn fn = encode_fn();
+    if (!fn) return ATTN_ERR_CUDA;
+    const cuuint64_t dims[4] = {64, 2, heads, rows > 0 ? rows : 1};
+    const cuuint64_t strides[3] = {128, 256, 256 * heads};
+    const cuuint32_t box[4] = {64, 2, 1, box_rows};
+    const cuuint32_t estr[4] = {1, 1, 1, 1};
+    CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void *>(base), dims,
+                    strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                    CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS ? ATTN_OK : ATTN_ERR_INVALID;
+}
+
 namespace {
 
 __global__ void wait_probe_kernel(uint64_t limit_ns) {

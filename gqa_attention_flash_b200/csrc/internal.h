@@ -20,6 +20,11 @@ attn_status_t make_tmap_bf16_3d(CUtensorMap *map, const void *base, uint64_t D, 
 attn_status_t make_tmap_bf16_paged(CUtensorMap *map, const void *base, uint64_t D, uint64_t heads,
                                    uint64_t rows, uint32_t box_rows);
 
+// The same cache with D = 128 viewed as (rows, heads, 2, 64): one (64, 2, 1, box_rows) box
+// copies both 64-column halves of box_rows rows, stored row by row (half 0, half 1).
+attn_status_t make_tmap_bf16_paged_wide(CUtensorMap *map, const void *base, uint64_t heads,
+                                        uint64_t rows, uint32_t box_rows);
+
 struct FwdArgs {
     void *O;
     const void *Q, *K, *V;
