@@ -15,7 +15,8 @@ Each draw runs through the C ABI and is compared with the oracle:
 - split-KV decode with random lengths and split counts;
 - the backward's dQ, dK, dV (tolerance as in test_gpu_bwd);
 - flex_attention! with a random score mod and mask mod, paged decode over random
-  block sizes and pools, and BlockMask-only calls on the block-sparse kernel.
+  block sizes and pools, and BlockMask-only calls on the block-sparse kernel;
+- larger forward draws (up to 8192 rows and keys) on sampled rows.
 
 The seeds are fixed, so every run checks the same configurations."""
 import math
@@ -278,3 +279,26 @@ def test_block_sparse_random_config(orc, seed):
     compare(O, L, Or, Lr, what=what)
     empty = torch.from_numpy(np.isneginf(Lr))
     assert torch.all(O.view(torch.int16)[empty] == 0), what
+
+
+LARGE_SEEDS = list(range(8000, 8016))
+
+
+@pytest.mark.parametrize("seed", LARGE_SEEDS)
+def test_forward_random_large_config(orc, seed):
+    """Larger draws (up to 8192 rows and keys, 32 query heads): enough work items that the
+    persistent CTAs take over several in turn.  The oracle checks sampled rows: tile edges,
+    the ends of the lengths and random rows, for every batch and head."""
+    from gpu_common import sample_rows
+    rng = np.random.default_rng(seed)
+    c = draw_prefill(rng, max_rows=8192, max_keys=8192, max_hq=32)
+    Q, K, V = W.random_prefill(seed, c["B"], c["Hq"], c["Hkv"], c["Sq"], c["Sk"], c["D"])
+    kl = None if c["k_lengths"] is None else torch.from_numpy(c["k_lengths"])
+    ql = None if c["q_lengths"] is None else torch.from_numpy(c["q_lengths"])
+    scale = 1.0 / math.sqrt(c["D"])
+    O, L = gpu_prefill(Q, K, V, scale, c["causal"], c["window"], c["input_pos"], kl, ql)
+    extra = [] if ql is None else [int(x) + d for x in ql.tolist() for d in (-1, 0)]
+    rows = sample_rows(c["Sq"], seed, n_random=24, extra=extra)
+    Or, Lr = oracle_prefill(orc, Q, K, V, scale, c["causal"], c["window"], c["input_pos"], kl, ql,
+                            rows=rows)
+    compare(O, L, Or, Lr, rows=rows, what=describe(c))
