@@ -8,7 +8,11 @@
 //
 // Work item: a pair of 128-row query tiles of one (query head, batch).  The grid
 // has one CTA per item, in launch order heaviest causal pairs first with the
-// query heads of one KV group adjacent, but the kernel is persistent: a running
+// query heads of one KV group adjacent.  When every item does the same work (no
+// causal mask, no window) and the last round of items would fill at most half of
+// the SMs, those last pairs run as two single-tile items each, so that round is
+// twice as wide (64x64-token image workload: 0.305 -> 0.294 ms, bitwise the same).
+// The kernel is persistent: a running
 // CTA takes over the items of CTAs not yet launched (cluster launch control), so
 // about one CTA per SM runs and the next item's Q and first K/V tiles load and its
 // first S products run while the current item finishes.  The two query tiles of
@@ -107,6 +111,7 @@ struct FwdParams {
     const int32_t *k_lengths;
     const int32_t *q_lengths;
     int B, Hq, Hkv, Sq, Sk, group, n_pairs;
+    int n_split;       // the last n_split pair items run as two single-tile items each
     float scale_log2;  // scale * log2(e)
     int causal, window, input_pos;
     uint64_t wait_limit_ns;
@@ -169,6 +174,8 @@ __device__ __forceinline__ float neg_inf() { return __int_as_float(0xff800000); 
 // the KV tiles they see.
 struct FwdItem {
     int pair, hq, b, hkv;
+    int qt0;                 // query tile of the item's tile 0 (tile 1 is qt0 + 1)
+    bool single;             // one query tile only (a split pair): tile 1 is not the item's
     int k_end, q_end;
     int lo0, hi0, lo1, hi1;  // KV tiles [lo_t, hi_t) that query tile t sees
     int ql0, ql1;            // last valid row of query tile t
@@ -186,11 +193,22 @@ __device__ __forceinline__ bool item_uses(const FwdItem &it, int t, int u) {
 // visible KV tile range of each query tile (whole-tile skipping).
 template <int kMode>
 __device__ __forceinline__ void fwd_item(const FwdParams &p, int w, FwdItem &it, bool report) {
+    // The last n_split pair items of the launch order are split in two: item
+    // n_full + 2 x + h is query tile h of pair item n_full + x.
+    const int n_full = p.n_pairs * p.Hq * p.B - p.n_split;
+    int half = 0;
+    it.single = false;
+    if (w >= n_full) {
+        half = (w - n_full) & 1;
+        w = n_full + ((w - n_full) >> 1);
+        it.single = true;
+    }
     it.hq = w % p.Hq;
     w /= p.Hq;
     it.b = w % p.B;
     w /= p.B;
     it.pair = p.n_pairs - 1 - w;
+    it.qt0 = it.pair * kTiles + half;
     it.hkv = it.hq / p.group;
     int k_end = p.Sk, q_end = p.Sq;
     if (p.k_lengths) {
@@ -214,9 +232,9 @@ __device__ __forceinline__ void fwd_item(const FwdParams &p, int w, FwdItem &it,
     // Tile t (0, 1) covers rows [q0_t, q0_t + 128) and sees KV tiles [lo_t, hi_t).
 #pragma unroll
     for (int t = 0; t < kTiles; ++t) {
-        const int q0 = (it.pair * kTiles + t) * BM;
+        const int q0 = (it.qt0 + t) * BM;
         int lo_t = 0, hi_t = 0, qlast = q0;
-        if (q0 < q_end && k_end > 0) {
+        if (q0 < q_end && k_end > 0 && !(t == 1 && it.single)) {
             qlast = min(q0 + BM - 1, q_end - 1);
             long long hi = k_end;
             if (p.causal) hi = min(hi, (long long)p.input_pos + qlast + 1);
@@ -313,9 +331,9 @@ __global__ void __launch_bounds__(kThreads, 1)
                 const int u = base + lane;
                 uint32_t e = 0;
                 if (u < it.u_hi) {
-                    const uint32_t s0 = item_uses(it, 0, u) ? flex_states(p, bm, it.pair * kTiles, u) : 0u;
+                    const uint32_t s0 = item_uses(it, 0, u) ? flex_states(p, bm, it.qt0, u) : 0u;
                     const uint32_t s1 =
-                        item_uses(it, 1, u) ? flex_states(p, bm, it.pair * kTiles + 1, u) : 0u;
+                        item_uses(it, 1, u) ? flex_states(p, bm, it.qt0 + 1, u) : 0u;
                     if (s0 | s1) e = static_cast<uint32_t>(u) | (s0 << 16) | (s1 << 24);
                 }
                 const uint32_t vote = __ballot_sync(0xffffffffu, e != 0);
@@ -399,7 +417,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 const int n_load = n_loads(it);
                 auto load_q = [&](int t) -> bool {
                     // checked build: the query tile lies inside Q
-                    if (!in_range(box_ok(0, (it.pair * kTiles + t) * BM, it.b * p.Hq + it.hq, D, p.Sq,
+                    if (!in_range(box_ok(0, (it.qt0 + t) * BM, it.b * p.Hq + it.hq, D, p.Sq,
                                          (long long)p.B * p.Hq, BM) &&
                                       it.pair >= 0 && it.pair < p.n_pairs,
                                   p.status, abort_flag))
@@ -411,7 +429,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                     mbar_arrive_expect_tx(bar(C::BAR_QFULL + slot), C::Q_BYTES);
                     for (int c = 0; c < C::NBOX; ++c)
                         tma_load_3d_hint(sbase + C::OFF_Q + slot * C::Q_BYTES + c * C::BOX, &tmQ,
-                                         bar(C::BAR_QFULL + slot), c * 64, (it.pair * kTiles + t) * BM,
+                                         bar(C::BAR_QFULL + slot), c * 64, (it.qt0 + t) * BM,
                                          it.b * p.Hq + it.hq, pol_q);
                     ++qi;
                     return true;
@@ -616,8 +634,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         uint32_t n_it = 0;  // S_t tiles of the previous items (S_FULL / O_DONE phases)
         uint32_t gi = 0;    // ring entries of the previous items
         for (int k = 0;; ++k) {
-            const int row = (it.pair * kTiles + t) * BM + r;
-            const int q0 = (it.pair * kTiles + t) * BM;
+            const int row = (it.qt0 + t) * BM + r;
+            const int q0 = (it.qt0 + t) * BM;
             const long long pos = (long long)p.input_pos + row;  // absolute position
             // this tile's range, selected without runtime-indexed arrays
             const int my_lo = t ? it.lo1 : it.lo0;
@@ -829,7 +847,8 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
 
             // step a8: epilogue
-            const bool row_in = row < p.Sq;
+            // a split pair's other tile belongs to the other single-tile item
+            const bool row_in = row < p.Sq && !(t == 1 && it.single);
             bool have = ok && n_done > 0;
             if (have && !warp_wait(bar_o, (n_it + n_done - 1) & 1, abort_flag, p.wait_limit_ns,
                                    p.status))
@@ -923,6 +942,19 @@ attn_status_t launch_fwd_d(const FwdArgs &a, cudaStream_t stream) {
     p.Sk = a.Sk;
     p.group = a.Hq / a.Hkv;
     p.n_pairs = (a.Sq + kTiles * BM - 1) / (kTiles * BM);
+    p.n_split = 0;
+    if (!kList && !a.causal && a.window == 0) {
+        // Items of equal work: when the last round of CTAs would be at most half full,
+        // its pair items run as single-tile items instead, filling it twice as wide.
+        int dev = 0, n_sm = 0;
+        if (cudaGetDevice(&dev) == cudaSuccess &&
+            cudaDeviceGetAttribute(&n_sm, cudaDevAttrMultiProcessorCount, dev) == cudaSuccess &&
+            n_sm > 0) {
+            const long long items = (long long)p.n_pairs * a.Hq * a.B;
+            const long long rem = items % n_sm;
+            if (items > n_sm && 2 * rem <= n_sm) p.n_split = static_cast<int>(rem);
+        }
+    }
     p.scale_log2 = a.scale * 1.4426950408889634f;
     p.causal = a.causal;
     p.window = a.window;
@@ -941,7 +973,7 @@ attn_status_t launch_fwd_d(const FwdArgs &a, cudaStream_t stream) {
     p.n_qb = (a.Sq + 63) / 64;
     p.n_kb = (a.Sk + 63) / 64;
     if (!p.status) return ATTN_ERR_CUDA;
-    const long long grid = (long long)p.n_pairs * a.Hq * a.B;
+    const long long grid = (long long)p.n_pairs * a.Hq * a.B + p.n_split;
     if (grid == 0) return ATTN_OK;
     if (grid > 0x7fffffffll) return ATTN_ERR_INVALID;
     attn_fwd_kernel<D, kMode, kList>
