@@ -95,14 +95,18 @@ def _tensor(t, name, dtype, shape):
 def _same_device(**tensors):
     """Every given tensor on the current CUDA device (the one whose stream the
     kernels are launched on)."""
+    cur = None
     for name, t in tensors.items():
         if t is None:
             continue
-        if not t.is_cuda:
+        idx = t.get_device()
+        if idx < 0:
             raise ValueError(f"{name} must be a CUDA tensor, got device {t.device}")
-        if t.device.index != torch.cuda.current_device():
+        if cur is None:
+            cur = torch.cuda.current_device()
+        if idx != cur:
             raise ValueError(f"{name} is on {t.device}, but the current device is "
-                             f"cuda:{torch.cuda.current_device()}")
+                             f"cuda:{cur}")
 
 
 def _check_prefill(O, Q, K, V, LSE, k_lengths, q_lengths):
