@@ -328,6 +328,12 @@ __global__ void __launch_bounds__(kThreads, 1)
         *abort_flag = 0;
         fence_mbar_init();
     }
+    // Programmatic dependent launch: the launch and the set-up above overlap the
+    // previous kernel on the stream; every global read or write below comes after
+    // that kernel has finished.  The next kernel may start its own set-up at once
+    // (its wait covers all of this grid).
+    asm volatile("griddepcontrol.wait;" ::: "memory");
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
     if constexpr (kList) {
         fwd_item<kMode>(p, blockIdx.x, it, false);
         // The KV tiles this CTA visits: inside a query tile's analytic range and
@@ -992,8 +998,18 @@ attn_status_t launch_fwd_d(const FwdArgs &a, cudaStream_t stream) {
     const long long grid = (long long)p.n_pairs * a.Hq * a.B + p.n_split;
     if (grid == 0) return ATTN_OK;
     if (grid > 0x7fffffffll) return ATTN_ERR_INVALID;
-    attn_fwd_kernel<D, kMode, kList>
-        <<<static_cast<unsigned>(grid), kThreads, kSmem, stream>>>(tq, tk, tv, p);
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(static_cast<unsigned>(grid), 1, 1);
+    cfg.blockDim = dim3(kThreads, 1, 1);
+    cfg.dynamicSmemBytes = kSmem;
+    cfg.stream = stream;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    if (cudaLaunchKernelEx(&cfg, attn_fwd_kernel<D, kMode, kList>, tq, tk, tv, p) != cudaSuccess)
+        return ATTN_ERR_CUDA;
     return cudaGetLastError() == cudaSuccess ? ATTN_OK : ATTN_ERR_CUDA;
 }
 
