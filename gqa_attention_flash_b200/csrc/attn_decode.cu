@@ -126,6 +126,12 @@ __global__ void __launch_bounds__(kDecThreads)
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
 
+    // Programmatic dependent launch: every global read or write below comes after
+    // the previous kernel on the stream has finished; the combine may launch at
+    // once (its own wait covers all of this grid).
+    asm volatile("griddepcontrol.wait;" ::: "memory");
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+
     int len = p.lengths[b];
     if (len > p.S_cap) {
         if (threadIdx.x == 0 && split == 0 && hkv == 0) record_status(p.status, ATTN_ERR_DEVICE_BOUNDS);
@@ -427,6 +433,9 @@ __global__ void __launch_bounds__(128)
     constexpr int WS = DecCfg<D>::WS_STRIDE;
     const int idx = blockIdx.x * 4 + (threadIdx.x >> 5);
     const int lane = threadIdx.x & 31;
+    // the split kernel's partials are complete and visible after this wait
+    asm volatile("griddepcontrol.wait;" ::: "memory");
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
     if (idx >= BH) return;
     const float *part = ws + (long long)idx * n_splits * WS;
     float M = neg_inf();
@@ -505,12 +514,27 @@ attn_status_t launch_decode_d(const DecodeArgs &a, cudaStream_t stream) {
     p.box_rows = static_cast<int>(box_rows);
     p.block_shift = 0;
     while (kPaged && (1 << p.block_shift) < a.block_size) ++p.block_shift;
-    dim3 grid(a.n_splits, a.Hkv, a.B);
-    decode_split_kernel<D, kPaged><<<grid, kDecThreads, C::SMEM_BYTES, stream>>>(tk, tv, p);
-    if (cudaGetLastError() != cudaSuccess) return ATTN_ERR_CUDA;
+    // Both kernels are launched with programmatic dependent launch (each waits for
+    // its predecessor on the stream before touching global memory).
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(a.n_splits, a.Hkv, a.B);
+    cfg.blockDim = dim3(kDecThreads, 1, 1);
+    cfg.dynamicSmemBytes = C::SMEM_BYTES;
+    cfg.stream = stream;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    if (cudaLaunchKernelEx(&cfg, decode_split_kernel<D, kPaged>, tk, tv, p) != cudaSuccess)
+        return ATTN_ERR_CUDA;
     const int BH = a.B * a.Hq;
-    decode_combine_kernel<D><<<(BH + 3) / 4, 128, 0, stream>>>(static_cast<__nv_bfloat16 *>(a.O),
-                                                                 a.workspace, BH, a.n_splits);
+    cfg.gridDim = dim3((BH + 3) / 4, 1, 1);
+    cfg.blockDim = dim3(128, 1, 1);
+    cfg.dynamicSmemBytes = 0;
+    if (cudaLaunchKernelEx(&cfg, decode_combine_kernel<D>, static_cast<__nv_bfloat16 *>(a.O),
+                           static_cast<const float *>(a.workspace), BH, a.n_splits) != cudaSuccess)
+        return ATTN_ERR_CUDA;
     return cudaGetLastError() == cudaSuccess ? ATTN_OK : ATTN_ERR_CUDA;
 }
 
