@@ -146,6 +146,11 @@ __global__ void __launch_bounds__(kSpThreads, 2)
         *abort_flag = 0;
         fence_mbar_init();
     }
+    // Programmatic dependent launch: launch and set-up overlap the previous kernel
+    // (the block scores that write the mask); every global access below follows
+    // its completion.
+    asm volatile("griddepcontrol.wait;" ::: "memory");
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
     if (warp == kSpWarpTma) {
         // The key blocks either query block of the tile keeps, in order (ballot
         // compaction, 32 blocks per round).
@@ -495,8 +500,18 @@ attn_status_t launch_bsparse_d(const FwdArgs &a, cudaStream_t stream) {
     const long long grid = (long long)p.n_qt * a.Hq * a.B;
     if (grid == 0) return ATTN_OK;
     if (grid > 0x7fffffffll) return ATTN_ERR_INVALID;
-    attn_fwd_bsparse_kernel<D><<<static_cast<unsigned>(grid), kSpThreads, C::SMEM_BYTES, stream>>>(
-        tq, tk, tv, p);
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(static_cast<unsigned>(grid), 1, 1);
+    cfg.blockDim = dim3(kSpThreads, 1, 1);
+    cfg.dynamicSmemBytes = C::SMEM_BYTES;
+    cfg.stream = stream;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    if (cudaLaunchKernelEx(&cfg, attn_fwd_bsparse_kernel<D>, tq, tk, tv, p) != cudaSuccess)
+        return ATTN_ERR_CUDA;
     return cudaGetLastError() == cudaSuccess ? ATTN_OK : ATTN_ERR_CUDA;
 }
 

@@ -330,6 +330,8 @@ __global__ void __launch_bounds__(128) rbs_scores_kernel(const ScoreParams p) {
     // query block is an input of the call and is staged while that grid finishes;
     // centroids, radii and beta are read only after it has completed.
     asm volatile("griddepcontrol.wait;" ::: "memory");
+    // the block-sparse attention that reads this mask may start its set-up now
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
     if (!p.beta) {
         // beta of the head's key blocks from its radii (rbs_beta_kernel's rule, here
         // for nkb <= 64 so that the estimator needs no separate sorting launch)
